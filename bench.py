@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Throughput of block-causal ReLU linear attention at 720p on B200 (one JSON line on rank 0).
+
+Workload (one "step"): the 720p block-causal prefill, B=1, H=20, D=128, 920 tokens per latent
+frame (23 x 40), blocks of 3 frames = 2760 tokens, 20 blocks = 55,200 tokens; bf16 q, k, v drawn
+N(0, 1) with numpy's seeded generator (seed = rank), fp32 accumulation, eps = 1e-6, final fp32
+cache written. One step is one call of sv_block_causal_attn: state reduction -> prefix scan ->
+output GEMM, i.e. every step of the hot path. Inputs (565 MB per step) are larger than the 126 MB
+L2, so L2 is not flushed between steps.
+
+  python bench.py [--gpus N --steps K --warmup W]        our CUDA path (torchrun for N > 1)
+  python bench.py --impl reference [...]                 the fp64 CPU oracle on the host cores
+
+With N > 1 every rank runs its own independent prefill (weak scaling, no data-path collective);
+the timed region is bracketed by barriers and the reported time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, H, N, D, L = 1, 20, 55200, 128, 2760
+EPS = 1e-6
+METRIC = "block-causal linear-attn tokens·heads/s at 720p; HBM GB/s & roofline fraction"
+UNIT = "tokens*heads/s"
+WORKLOAD = {
+    "workload": "720p block-causal prefill: B=1 H=20 N=55200 (20 blocks x 2760 tokens = 3 latent frames "
+                "x 23x40) D=128, bf16 q/k/v ~ N(0,1), fp32 accumulation, eps=1e-6, final fp32 cache out",
+    "B": B, "H": H, "N": N, "D": D, "block_len": L,
+    "seed": "rank",
+    "l2": "inputs 565 MB per step > 126 MB L2; not flushed",
+}
+ALG_BYTES_PER_TOKHEAD = 4 * D * 2              # read q, k, v once, write o once (bf16)
+ALG_FLOPS_PER_TOKHEAD = 4 * D * D + 4 * D       # state 2D^2 + z D, numerator 2D^2 + den 2D + div D
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML, the source nvidia-smi reads)
+# ----------------------------------------------------------------------------------------------
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - NVML missing
+            self._nv = None
+            self.error = str(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                bits = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in _REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------------------------
+# the oracle on the host cores (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_rate(q, k, v, budget_s: float, max_heads: int | None = None):
+    """Time the fp64 oracle (as it stands) head by head on the stored inputs until budget_s elapse.
+    Returns (tokens*heads per second, heads done, tokens per head, seconds)."""
+    import oracle
+    from block_causal_linear_relu_b200.inputs import to_f64
+
+    done, t0 = 0, time.perf_counter()
+    limit = max_heads if max_heads is not None else H
+    while done < limit:
+        h = done % H
+        qh, kh, vh = (to_f64(x[:, h:h + 1], "bf16") for x in (q, k, v))
+        oracle.block_causal_attn(qh, kh, vh, L, EPS)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done * N / dt, done, N, dt
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    from block_causal_linear_relu_b200.inputs import draw_qkv
+
+    q, k, v = draw_qkv((B, H, N, D), 0, "bf16")
+    # one warm-up head sizes the per-step sample so that the whole run stays within a few minutes
+    r0, _, _, t_head = oracle_rate(q, k, v, 0.0, max_heads=1)
+    per_step_budget = max(0.0, min(t_head * H, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_rate(q, k, v, 0.0, max_heads=1)
+    tot_heads, tot_s = 0, 0.0
+    for _ in range(args.steps):
+        _, nh, _, dt = oracle_rate(q, k, v, per_step_budget)
+        tot_heads, tot_s = tot_heads + nh, tot_s + dt
+    value = tot_heads * N / tot_s
+    cores = _blas_threads()
+    sample = (f"fp64 numpy oracle (state form), {tot_heads} heads x {N} tokens of the seed-0 720p prefill "
+              f"over {args.steps} steps (each step >= 1 head, bounded)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": WORKLOAD,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------------------
+# our CUDA path
+# ----------------------------------------------------------------------------------------------
+def _source_sha():
+    h = hashlib.sha256()
+    for f in ("sv_kernels.cu", "sv_ptx.cuh", "sv_geometry.h"):
+        with open(os.path.join(ROOT, "block_causal_linear_relu_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        ent = j.get(kernel)
+        if ent and ent.get("source_sha") == _source_sha():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+
+    import block_causal_linear_relu_b200 as sv
+    from block_causal_linear_relu_b200.inputs import draw_qkv
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)) if world > 1 else 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sv.load()
+    hbm_gbs, tf_burst, tf_sust, peak_src = peaks()
+
+    qs, ks, vs = draw_qkv((B, H, N, D), rank, "bf16")
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to_dev(qs), to_dev(ks), to_dev(vs)
+    o = torch.empty_like(q)
+    S_out = torch.zeros(B, H, D, D, device=dev)
+    z_out = torch.zeros(B, H, D, device=dev)
+    stream = torch.cuda.current_stream()
+    ws = sv.make_workspace(sv.SV_OP_BLOCK_CAUSAL_ATTN, q, L)
+
+    def step():
+        sv.sv_block_causal_attn(q, k, v, L, o=o, eps=EPS, S_out=S_out, z_out=z_out, ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    # per-step stage events (recorded between the three kernels by the library's timing hook)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            sv.sv_profile_events(evs[i])
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    sv.sv_profile_events(None)
+    barrier()
+    torch.cuda.synchronize()
+    ms = t_start.elapsed_time(t_end)
+    st_ms = sum(r[0].elapsed_time(r[1]) for r in evs) / args.steps
+    sc_ms = sum(r[1].elapsed_time(r[2]) for r in evs) / args.steps
+    ou_ms = sum(r[2].elapsed_time(r[3]) for r in evs) / args.steps
+    if world > 1:
+        t = torch.tensor([ms, st_ms, sc_ms, ou_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, st_ms, sc_ms, ou_ms = t.tolist()
+    if ws.status() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout")
+
+    tokheads = B * H * N
+    value = world * tokheads * args.steps / (ms / 1e3)
+    ms_step = ms / args.steps
+
+    # end to end through the public API: pinned host inputs -> device -> call -> o back to host
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+        qh, kh, vh = pin(qs), pin(ks), pin(vs)
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = t.item()
+        e2e = {"value": world * tokheads * n_e2e / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2,
+               "steps": n_e2e, "ms_per_step": ems / n_e2e}
+
+    if rank != 0:
+        return 0
+    io_bytes_half = 2 * tokheads * D * 2  # state kernel reads k, v; output kernel reads q, writes o
+    kernels = {"state_reduce": st_ms, "prefix_scan": sc_ms, "out_gemm": ou_ms}
+    dom = "state_reduce" if st_ms >= ou_ms else "out_gemm"
+    dom_ms = kernels[dom]
+    achieved = io_bytes_half / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved / hbm_gbs, "traffic": _traffic(dom),
+                "peak_source": f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6650 GB/s",
+                "alg_bytes_per_launch": io_bytes_half, "avg_launch_ms": dom_ms}
+    step_bytes = tokheads * ALG_BYTES_PER_TOKHEAD
+    step_flops = tokheads * ALG_FLOPS_PER_TOKHEAD
+    t_roof = max(step_bytes / (hbm_gbs * 1e9), step_flops / (tf_burst * 1e12))
+    step_roof = {"alg_bytes": step_bytes, "alg_flops": step_flops, "t_roof_us": t_roof * 1e6,
+                 "t_meas_us": ms_step * 1e3, "frac": t_roof / (ms_step / 1e3),
+                 "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                 "achieved_tflops": step_flops / (ms_step / 1e3) / 1e12}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, nh, ntok, secs = oracle_rate(qs, ks, vs, args.cpu_budget)
+        cpu = {"value": rate, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+               "sample": f"fp64 numpy oracle (state form) on {nh} of {H} heads x {ntok} tokens of this "
+                         f"workload, {secs:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": WORKLOAD,
+        "roofline": roofline, "step_roofline": step_roof,
+        "kernels_ms": kernels, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+        "gpu_launches": 3 * args.steps, "impl": "ours",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))))
+        try:
+            return run_ours(args, rank, world)
+        finally:
+            dist.destroy_process_group()
+    return run_ours(args, rank, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

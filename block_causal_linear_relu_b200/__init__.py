@@ -1,0 +1,27 @@
+"""ReLU-kernel linear attention (bidirectional and block-causal with a constant-memory cache)
+for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libsvlinattn.so`` (hand-written CUDA, C ABI declared in
+``include/svlinattn.h``); this package is its thin ctypes binding plus a seeded input generator.
+"""
+
+from ._native import (  # noqa: F401
+    EXPORTS,
+    SV_BF16,
+    SV_F32,
+    SV_OP_BLOCK_CAUSAL_ATTN,
+    SV_OP_BLOCK_STATE_UPDATE,
+    SV_OP_CACHE_STEP,
+    SV_OP_LINATTN_FWD,
+    SvError,
+    Workspace,
+    lib_path,
+    load,
+    make_workspace,
+    sv_block_causal_attn,
+    sv_block_state_update,
+    sv_cache_step,
+    sv_linattn_fwd,
+    sv_profile_events,
+    workspace_bytes,
+)

@@ -1,0 +1,210 @@
+"""ctypes binding of libsvlinattn.so: argument marshalling only, every step runs in the library.
+
+Functions carry the C entry points' names. Tensors are torch CUDA tensors (PyTorch supplies device
+memory and streams); outputs and the workspace are allocated here when the caller gives none.
+There is no fallback: if the shared library is missing or the device is not a B200 the call
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsvlinattn.so")
+_lib = None
+_lock = threading.Lock()
+
+SV_OK, SV_ERR_INVALID_ARG, SV_ERR_UNSUPPORTED, SV_ERR_CUDA, SV_ERR_TIMEOUT = range(5)
+SV_BF16, SV_F32 = 0, 1
+SV_OP_LINATTN_FWD, SV_OP_BLOCK_STATE_UPDATE, SV_OP_BLOCK_CAUSAL_ATTN, SV_OP_CACHE_STEP = range(4)
+
+#: every symbol include/svlinattn.h declares
+EXPORTS = (
+    "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_linattn_fwd",
+    "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_profile_events", "sv_last_error",
+    "sv_version",
+)
+
+
+class SvError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"sv status {status}: {msg}")
+        self.status = status
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load libsvlinattn.so (built in-tree by block_causal_linear_relu_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m block_causal_linear_relu_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, sz, i, f, u32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
+        lib.sv_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        lib.sv_workspace_bytes.restype = sz
+        lib.sv_workspace_init.argtypes = [vp, sz, vp]
+        lib.sv_workspace_init.restype = i
+        lib.sv_device_status.argtypes = [vp, vp, u32p]
+        lib.sv_device_status.restype = i
+        lib.sv_linattn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+        lib.sv_linattn_fwd.restype = i
+        lib.sv_block_state_update.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, sz, vp]
+        lib.sv_block_state_update.restype = i
+        lib.sv_block_causal_attn.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp, vp, sz, vp]
+        lib.sv_block_causal_attn.restype = i
+        lib.sv_cache_step.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, vp, vp, i, vp, sz, vp]
+        lib.sv_cache_step.restype = i
+        lib.sv_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
+        lib.sv_profile_events.restype = i
+        lib.sv_last_error.argtypes = []
+        lib.sv_last_error.restype = ctypes.c_char_p
+        lib.sv_version.argtypes = []
+        lib.sv_version.restype = i
+        _lib = lib
+        return lib
+
+
+def _check(status: int):
+    if status != SV_OK:
+        raise SvError(status, load().sv_last_error().decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SV_BF16
+    if t.dtype == torch.float32:
+        return SV_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32 expected")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _qkv(*ts):
+    ref = ts[0]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, N, D]")
+        if t.dim() != 4 or t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+            raise ValueError("q, k, v, o must share shape [B, H, N, D], dtype and device")
+    return ref.shape
+
+
+def workspace_bytes(op: int, B: int, H: int, N: int, D: int, block_len: int, dtype: int, device=None) -> int:
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        n = load().sv_workspace_bytes(op, B, H, N, D, block_len, dtype)
+    if n == 0:
+        raise SvError(SV_ERR_INVALID_ARG, load().sv_last_error().decode())
+    return int(n)
+
+
+class Workspace:
+    """Caller-owned device scratch: a 256-byte aligned view into a torch uint8 buffer."""
+
+    def __init__(self, nbytes: int, device, stream=None):
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.view = self.buf[off:off + nbytes]
+        self.nbytes = nbytes
+        _check(load().sv_workspace_init(ctypes.c_void_p(self.view.data_ptr()), nbytes, _stream(stream)))
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.view.data_ptr())
+
+    def status(self, stream=None) -> int:
+        code = ctypes.c_uint32(0)
+        st = load().sv_device_status(self.ptr, _stream(stream), ctypes.byref(code))
+        if st not in (SV_OK, SV_ERR_TIMEOUT):
+            _check(st)
+        return int(code.value)
+
+
+def make_workspace(op: int, q_like: torch.Tensor, block_len: int | None = None, stream=None) -> Workspace:
+    B, H, N, D = q_like.shape
+    n = workspace_bytes(op, B, H, N, D, block_len if block_len is not None else N, _dt(q_like), q_like.device)
+    return Workspace(n, q_like.device, stream)
+
+
+def _ws(ws, op, q_like, block_len, stream):
+    return ws if ws is not None else make_workspace(op, q_like, block_len, stream)
+
+
+def sv_linattn_fwd(q, k, v, o=None, eps: float = 1e-6, ws: Workspace | None = None, stream=None):
+    """Bidirectional ReLU linear attention; returns o."""
+    B, H, N, D = _qkv(q, k, v)
+    o = torch.empty_like(q) if o is None else o
+    _qkv(q, o)
+    ws = _ws(ws, SV_OP_LINATTN_FWD, q, None, stream)
+    _check(load().sv_linattn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, ws.ptr, ws.nbytes,
+                                 _stream(stream)))
+    return o
+
+
+def sv_block_causal_attn(q, k, v, block_len: int, o=None, eps: float = 1e-6, S_in=None, z_in=None, S_out=None,
+                         z_out=None, ws: Workspace | None = None, stream=None):
+    """Block-causal prefill; returns o (S_out/z_out are written in place when given)."""
+    B, H, N, D = _qkv(q, k, v)
+    o = torch.empty_like(q) if o is None else o
+    _qkv(q, o)
+    for t in (S_in, z_in, S_out, z_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != q.device):
+            raise ValueError("S/z must be contiguous float32 tensors on q's device")
+    ws = _ws(ws, SV_OP_BLOCK_CAUSAL_ATTN, q, block_len, stream)
+    _check(load().sv_block_causal_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, int(block_len), _dt(q), eps,
+                                       _ptr(S_in), _ptr(z_in), _ptr(S_out), _ptr(z_out), ws.ptr, ws.nbytes,
+                                       _stream(stream)))
+    return o
+
+
+def sv_cache_step(q, k, v, S, z, commit: bool = True, o=None, eps: float = 1e-6, ws: Workspace | None = None,
+                  stream=None):
+    """One streaming block against the fp32 cache (S [B,H,D,D], z [B,H,D]); returns o."""
+    B, H, N, D = _qkv(q, k, v)
+    o = torch.empty_like(q) if o is None else o
+    _qkv(q, o)
+    if S.dtype != torch.float32 or z.dtype != torch.float32 or tuple(S.shape) != (B, H, D, D) or tuple(z.shape) != (B, H, D):
+        raise ValueError("cache must be float32 S [B,H,D,D] and z [B,H,D]")
+    ws = _ws(ws, SV_OP_CACHE_STEP, q, None, stream)
+    _check(load().sv_cache_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, _ptr(S), _ptr(z),
+                                1 if commit else 0, ws.ptr, ws.nbytes, _stream(stream)))
+    return o
+
+
+def sv_profile_events(events):
+    """Install (list of 4 torch.cuda.Event, already recorded once) or clear (None) the timing hook."""
+    if events is None:
+        _check(load().sv_profile_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(load().sv_profile_events(arr, 4))
+
+
+def sv_block_state_update(k, v, S, z, ws: Workspace | None = None, stream=None):
+    """S += ReLU(K)^T V, z += sum ReLU(k), in place."""
+    B, H, N, D = _qkv(k, v)
+    if S.dtype != torch.float32 or z.dtype != torch.float32 or tuple(S.shape) != (B, H, D, D) or tuple(z.shape) != (B, H, D):
+        raise ValueError("cache must be float32 S [B,H,D,D] and z [B,H,D]")
+    ws = _ws(ws, SV_OP_BLOCK_STATE_UPDATE, k, None, stream)
+    _check(load().sv_block_state_update(_ptr(k), _ptr(v), B, H, N, D, _dt(k), _ptr(S), _ptr(z), ws.ptr, ws.nbytes,
+                                        _stream(stream)))
+    return S, z

@@ -1,0 +1,44 @@
+// Internal launch interface between the C-ABI layer (sv_api.cu) and the kernels (sv_kernels.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sv_geometry.h"
+
+namespace sv {
+
+// Tensor maps of one [BH, N, D] bf16 tensor seen as blocks: `main` covers the blocks of length L,
+// `last` the shorter last block when N is not a multiple of L (else it repeats `main`).
+struct BlockMaps {
+  CUtensorMap main;
+  CUtensorMap last;
+};
+
+struct Bf16Launch {
+  BlockMaps q, k, v, o;     // q/k/v: 128-row load boxes; o: 32-row store boxes
+  const uint16_t* ptiles;   // workspace: bf16 prefix tiles (nseg x kPTileBytes)
+};
+
+// bf16 path
+cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials,
+                              uint32_t* status, cudaStream_t st);
+cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles,
+                            float eps, uint32_t* status, cudaStream_t st);
+// fp32 path
+cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, uint32_t* status,
+                             cudaStream_t st);
+cudaError_t launch_out_f32(const float* q, float* o, const Geom& g, const float* p32, float eps,
+                           uint32_t* status, cudaStream_t st);
+// both paths: combine partials, inclusive prefix over blocks, optional final cache
+cudaError_t launch_scan(const float* partials, const Geom& g, const float* S_in, const float* z_in,
+                        float* S_out, float* z_out, void* ptiles_bf16, float* p32, cudaStream_t st);
+
+size_t state_bf16_smem_bytes();
+size_t out_bf16_smem_bytes();
+size_t state_f32_smem_bytes();
+size_t out_f32_smem_bytes();
+cudaError_t set_kernel_attributes();
+
+}  // namespace sv

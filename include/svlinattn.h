@@ -1,0 +1,130 @@
+/*
+ * svlinattn — ReLU-kernel linear attention on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operation (SANA-Video, "Efficient Video Generation with Block Linear Diffusion
+ * Transformer"; talk at ICLR 2026, block KV cache passage, and the paper abstract, design (2)
+ * "Constant-Memory KV cache for Block Linear Attention"):
+ *
+ *     phi(x) = max(x, 0)                                  (feature map, elementwise)
+ *     S      = sum_j phi(k_j)^T v_j    [D x D]            (state: row = key feature d,
+ *     z      = sum_j phi(k_j)          [D]                         column = value feature e)
+ *     o_i    = phi(q_i) S / (phi(q_i) . z + eps)
+ *
+ * Linear attention keeps a state of fixed shape D x D whatever the sequence length. In the
+ * block-causal form a video is generated block by block: a block attends to itself
+ * (bidirectionally, it is diffused as a whole) and to the state summed over all previous blocks;
+ * after the block, its own state is added to that cache. The cache (S, z) therefore has constant
+ * size, B*H*D*(D+1) fp32 values, however many blocks have been generated.
+ *
+ * Conventions shared by every entry point
+ *  - q, k, v, o are DEVICE pointers to contiguous [B, H, N, D] tensors (row-major, D fastest),
+ *    element type `dt` (SV_BF16: bfloat16, SV_F32: float). o has the type of q. 16-byte aligned.
+ *  - S is a DEVICE pointer to fp32 [B, H, D, D] (S[b][h][d][e], d = key feature, e = value
+ *    feature), z a DEVICE pointer to fp32 [B, H, D]. 4-byte aligned. The cache is always fp32.
+ *  - ws is caller-owned DEVICE scratch of at least sv_workspace_bytes(...) bytes, 256-byte
+ *    aligned, zero-initialised once with sv_workspace_init before its first use. Its first
+ *    256 bytes hold a status word that the kernels raise when a bounded wait expires.
+ *    Calls that share one workspace must be ordered on the GPU (same stream, or synchronised).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *    Pointers stay owned by the caller; the library allocates nothing and keeps no state
+ *    between calls other than per-device kernel attributes.
+ *  - Supported sizes: B, H, N >= 1; SV_BF16: D in {64, 80, 96, 112, 128};
+ *    SV_F32: 1 <= D <= 128. eps must be finite and >= 0.
+ *  - Errors: every argument is checked on the host BEFORE anything is launched; a bad argument
+ *    returns SV_ERR_INVALID_ARG / SV_ERR_UNSUPPORTED and launches nothing. A failed launch returns
+ *    SV_ERR_CUDA. Device-side timeouts (SV_ERR_TIMEOUT) are reported by sv_device_status.
+ *    sv_last_error() gives a message for the calling thread's last non-OK status.
+ *  - NaN/Inf inputs propagate; nothing checks for them.
+ */
+#ifndef SVLINATTN_H
+#define SVLINATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SV_OK = 0,
+  SV_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size <= 0, workspace too small, bad eps */
+  SV_ERR_UNSUPPORTED = 2, /* D or dtype not supported, device is not sm_100 */
+  SV_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a launch failed */
+  SV_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (read through sv_device_status) */
+} sv_status;
+
+typedef enum { SV_BF16 = 0, SV_F32 = 1 } sv_dtype;
+
+typedef enum {
+  SV_OP_LINATTN_FWD = 0,
+  SV_OP_BLOCK_STATE_UPDATE = 1,
+  SV_OP_BLOCK_CAUSAL_ATTN = 2,
+  SV_OP_CACHE_STEP = 3
+} sv_op;
+
+typedef struct CUstream_st* sv_stream_t; /* same type as cudaStream_t */
+
+/* Bytes of workspace the call `op` needs for these sizes on the CURRENT device (the number of
+ * streaming multiprocessors enters the size). block_len is read only for
+ * SV_OP_BLOCK_CAUSAL_ATTN. Returns 0 for invalid sizes (see sv_last_error). */
+size_t sv_workspace_bytes(sv_op op, int B, int H, int N, int D, int block_len, sv_dtype dt);
+
+/* Zero the workspace's status word (asynchronous on `stream`). Call once after allocating. */
+sv_status sv_workspace_init(void* ws, size_t ws_bytes, sv_stream_t stream);
+
+/* Synchronise `stream`, read the workspace's status word and clear it. SV_OK if no kernel
+ * raised it; SV_ERR_TIMEOUT if a bounded wait expired (the word is then in *code, if given). */
+sv_status sv_device_status(void* ws, sv_stream_t stream, uint32_t* code);
+
+/* Bidirectional full-sequence linear attention (the Linear DiT layer: every token attends to
+ * every token of its (b, h) sequence; SANA-Video abstract, design (1) "Linear DiT"):
+ *     o_i = phi(q_i) S / (phi(q_i) . z + eps),  S, z summed over all N tokens. */
+sv_status sv_linattn_fwd(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                         sv_dtype dt, float eps, void* ws, size_t ws_bytes, sv_stream_t stream);
+
+/* Add a block's state to the cache in place (talk, block KV cache passage: the state is updated
+ * additively, the current block's contribution added to the previous cache):
+ *     S += phi(K)^T V,  z += sum_j phi(k_j)  over the N tokens of k, v ([B, H, N, D]). */
+sv_status sv_block_state_update(const void* k, const void* v, int B, int H, int N, int D, sv_dtype dt, float* S,
+                                float* z, void* ws, size_t ws_bytes, sv_stream_t stream);
+
+/* Block-causal prefill over a whole sequence cut into blocks of block_len tokens (the last block
+ * may be shorter). Token i of block c = floor(i / block_len) attends to every token of blocks
+ * 0..c plus the incoming cache:
+ *     P_c = S_in + sum_{c' <= c} S_c',  zP_c = z_in + sum_{c' <= c} z_c',
+ *     o_i = phi(q_i) P_c / (phi(q_i) . zP_c + eps).
+ * S_in/z_in (nullable: zero cache) is the cache before the sequence; S_out/z_out (nullable: not
+ * written) receives the cache after the last block. S_out may equal S_in (in-place update).
+ * block_len >= N is the bidirectional form. */
+sv_status sv_block_causal_attn(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                               int block_len, sv_dtype dt, float eps, const float* S_in, const float* z_in,
+                               float* S_out, float* z_out, void* ws, size_t ws_bytes, sv_stream_t stream);
+
+/* One streaming step of the constant-memory cache (talk, block-causal walkthrough: the block's
+ * output uses the cached state plus its own contribution; the new state is then cached): the
+ * N tokens of q, k, v form one block, o = attention of the block over (block + cache). If
+ * commit != 0 the cache then takes the block's state (S += phi(K)^T V, z += sum phi(k)); with
+ * commit == 0 S and z are left untouched (e.g. the intermediate denoising steps of a block). */
+sv_status sv_cache_step(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                        sv_dtype dt, float eps, float* S, float* z, int commit, void* ws, size_t ws_bytes,
+                        sv_stream_t stream);
+
+/* Optional timing hook for benchmarks. With events != NULL (n == 4 cudaEvent_t handles owned by
+ * the caller), the calling thread's following forward calls (sv_linattn_fwd, sv_block_causal_attn,
+ * sv_cache_step) record events[0] before the state-reduction kernel, events[1] after it,
+ * events[2] after the prefix scan and events[3] after the output kernel, on the call's stream.
+ * events == NULL (n ignored) removes the hook. Costs one cudaEventRecord per mark. */
+sv_status sv_profile_events(void* const* events, int n);
+
+/* Message for the calling thread's most recent non-OK status ("" if none). */
+const char* sv_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int sv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVLINATTN_H */

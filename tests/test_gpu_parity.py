@@ -1,0 +1,321 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded inputs.
+
+Tolerances (normwise max relative error, max|g - r| / max|r|, per output tensor):
+  bf16 I/O : 2e-2 on o;  fp32 I/O : 1e-4 on o.
+  fp32 cache (S, z) : 1e-4 for both dtypes -- the cache is accumulated in fp32 from exact
+  products of the stored inputs, so its error is fp32 summation error only.
+Small shapes are compared element by element in full; the full-size shapes that the bench times
+are compared on sampled heads and rows that the oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_causal_linear_relu_b200.inputs import draw_qkv, to_f64
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+TOL_CACHE = 1e-4
+EPS = 1e-6
+
+
+@pytest.fixture(scope="module")
+def sv():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from block_causal_linear_relu_b200 import build
+    build.build()
+    import block_causal_linear_relu_b200 as m
+    m.load()
+    return m
+
+
+def dev(x, dtype):
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def host(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def inputs(shape, seed, dtype):
+    q, k, v = draw_qkv(shape, seed, dtype)
+    return (q, k, v), tuple(to_f64(x, dtype) for x in (q, k, v))
+
+
+def run_bc(sv, qkv, dtype, L, **kw):
+    q, k, v = (dev(x, dtype) for x in qkv)
+    o = sv.sv_block_causal_attn(q, k, v, L, eps=EPS, **kw)
+    torch.cuda.synchronize()
+    return o
+
+
+# --------------------------------------------------------------------------------------------
+# config 0: fp32 [1, 2, 256, 32], 4 blocks x 64 tokens, eps 1e-6, both forms, 1e-4
+# --------------------------------------------------------------------------------------------
+def test_c0_fp32_block_causal_and_bidirectional(sv):
+    st, (q, k, v) = inputs((1, 2, 256, 32), 0, "f32")
+    S_out = torch.zeros(1, 2, 32, 32, device="cuda")
+    z_out = torch.zeros(1, 2, 32, device="cuda")
+    o = run_bc(sv, st, "f32", 64, S_out=S_out, z_out=z_out)
+    ref = oracle.bruteforce_masked(q, k, v, 64, EPS)
+    assert oracle.max_rel_err(host(o), ref) < TOL["f32"]
+    _, S_ref, z_ref = oracle.block_causal_attn(q, k, v, 64, EPS)
+    assert oracle.max_rel_err(host(S_out), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z_out), z_ref) < TOL_CACHE
+    qd, kd, vd = (dev(x, "f32") for x in st)
+    ob = sv.sv_linattn_fwd(qd, kd, vd, eps=EPS)
+    torch.cuda.synchronize()
+    assert oracle.max_rel_err(host(ob), oracle.bruteforce_masked(q, k, v, 256, EPS)) < TOL["f32"]
+
+
+@pytest.mark.parametrize("B,H,N,D,L", [(1, 2, 300, 32, 64), (2, 1, 97, 128, 40), (1, 3, 9, 7, 1),
+                                       (1, 1, 1000, 64, 1000), (1, 2, 513, 100, 129)])
+def test_fp32_shapes(sv, B, H, N, D, L):
+    st, (q, k, v) = inputs((B, H, N, D), 5, "f32")
+    o = run_bc(sv, st, "f32", L)
+    assert oracle.max_rel_err(host(o), oracle.block_causal_attn(q, k, v, L, EPS)[0]) < TOL["f32"]
+
+
+# --------------------------------------------------------------------------------------------
+# bf16 tensor-core path: several tiles, ragged tails, every supported D, degenerate blocks
+# --------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("B,H,N,D,L", [
+    (1, 2, 700, 128, 300),     # partial last block (100 tokens), block tails of 44 rows
+    (2, 3, 1000, 112, 1000),   # bidirectional, D = 112 (zero-filled feature tail)
+    (1, 2, 517, 64, 200),      # D = 64 (one feature atom)
+    (1, 1, 130, 80, 64),       # D = 80
+    (1, 2, 384, 96, 128),      # block = one tile exactly
+    (1, 1, 1, 128, 1),         # a single token
+    (1, 2, 5, 128, 1),         # block_len = 1: token-causal
+    (1, 1, 257, 128, 1000),    # block_len > N
+    (3, 5, 333, 128, 111),
+])
+def test_bf16_shapes(sv, B, H, N, D, L):
+    st, (q, k, v) = inputs((B, H, N, D), 1, "bf16")
+    o = run_bc(sv, st, "bf16", L)
+    err = oracle.max_rel_err(host(o), oracle.block_causal_attn(q, k, v, L, EPS)[0])
+    assert err < TOL["bf16"], err
+
+
+def test_bf16_many_tiles_per_cta(sv):
+    # 8 heads x 8 blocks of 2760 (last 680): ~8.6 tiles per CTA, CTAs cross segment boundaries
+    st, (q, k, v) = inputs((1, 8, 20000, 128), 2, "bf16")
+    S_out = torch.zeros(1, 8, 128, 128, device="cuda")
+    z_out = torch.zeros(1, 8, 128, device="cuda")
+    o = run_bc(sv, st, "bf16", 2760, S_out=S_out, z_out=z_out)
+    ref, S_ref, z_ref = oracle.block_causal_attn(q, k, v, 2760, EPS)
+    assert oracle.max_rel_err(host(o), ref) < TOL["bf16"]
+    assert oracle.max_rel_err(host(S_out), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z_out), z_ref) < TOL_CACHE
+
+
+def test_bf16_error_is_well_inside_tolerance(sv):
+    # the bf16 path's only rounding steps are the bf16 prefix operand and the bf16 output:
+    # the measured error should sit near 1e-3, an order below the 2e-2 bar
+    st, (q, k, v) = inputs((1, 4, 4000, 128), 3, "bf16")
+    o = run_bc(sv, st, "bf16", 1000)
+    err = oracle.max_rel_err(host(o), oracle.block_causal_attn(q, k, v, 1000, EPS)[0])
+    assert err < 5e-3, err
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_incoming_cache_and_in_place_update(sv, dtype):
+    B, H, N, D, L = 1, 3, 600, 128, 250
+    st, (q, k, v) = inputs((B, H, N, D), 4, dtype)
+    rng = np.random.default_rng(4)
+    S0 = rng.standard_normal((B, H, D, D)).astype(np.float32) * 30
+    z0 = np.abs(rng.standard_normal((B, H, D))).astype(np.float32) * 50
+    S = torch.from_numpy(S0).cuda()
+    z = torch.from_numpy(z0).cuda()
+    o = run_bc(sv, st, dtype, L, S_in=S, z_in=z, S_out=S, z_out=z)  # in place
+    ref, S_ref, z_ref = oracle.block_causal_attn(q, k, v, L, EPS, S0.astype(np.float64), z0.astype(np.float64))
+    assert oracle.max_rel_err(host(o), ref) < TOL[dtype]
+    assert oracle.max_rel_err(host(S), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_state_update(sv, dtype):
+    B, H, N, D = 2, 2, 777, 128
+    st, (_, k, v) = inputs((B, H, N, D), 6, dtype)
+    rng = np.random.default_rng(6)
+    S0 = rng.standard_normal((B, H, D, D)).astype(np.float32)
+    z0 = np.abs(rng.standard_normal((B, H, D))).astype(np.float32)
+    S = torch.from_numpy(S0).cuda()
+    z = torch.from_numpy(z0).cuda()
+    sv.sv_block_state_update(dev(st[1], dtype), dev(st[2], dtype), S, z)
+    torch.cuda.synchronize()
+    S_ref, z_ref = oracle.block_state_update(k, v, S0.astype(np.float64), z0.astype(np.float64))
+    assert oracle.max_rel_err(host(S), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_streaming_matches_prefill_and_oracle(sv, dtype):
+    B, H, D, L, nb = 1, 4, 128, 500, 6
+    st, (q, k, v) = inputs((B, H, nb * L, D), 7, dtype)
+    qd, kd, vd = (dev(x, dtype) for x in st)
+    S = torch.zeros(B, H, D, D, device="cuda")
+    z = torch.zeros(B, H, D, device="cuda")
+    ws = sv.make_workspace(sv.SV_OP_CACHE_STEP, qd[:, :, :L].contiguous())
+    outs = []
+    for c in range(nb):
+        sl = slice(c * L, (c + 1) * L)
+        qb, kb, vb = (x[:, :, sl].contiguous() for x in (qd, kd, vd))
+        S_before, z_before = S.clone(), z.clone()
+        o0 = sv.sv_cache_step(qb, kb, vb, S, z, commit=False, eps=EPS, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(S, S_before) and torch.equal(z, z_before)  # commit=0 leaves the cache
+        o1 = sv.sv_cache_step(qb, kb, vb, S, z, commit=True, eps=EPS, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(o0, o1)
+        outs.append(o1)
+    o = torch.cat(outs, dim=2)
+    ref, S_ref, z_ref = oracle.block_causal_attn(q, k, v, L, EPS)
+    assert oracle.max_rel_err(host(o), ref) < TOL[dtype]
+    assert oracle.max_rel_err(host(S), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
+    op = sv.sv_block_causal_attn(qd, kd, vd, L, eps=EPS)
+    torch.cuda.synchronize()
+    assert oracle.max_rel_err(host(op), host(o)) < TOL[dtype]
+    assert ws.status() == 0
+
+
+def test_nonpositive_query_rows_give_exact_zero(sv):
+    st, _ = inputs((1, 2, 300, 128), 8, "bf16")
+    q = st[0].copy()
+    q[0, 1, 5] |= np.uint16(0x8000)   # force every feature of token 5 (head 1) negative
+    q[0, 0, 299] = 0                  # all +0.0
+    o = run_bc(sv, (q, st[1], st[2]), "bf16", 128)
+    assert torch.count_nonzero(o[0, 1, 5]) == 0 and torch.count_nonzero(o[0, 0, 299]) == 0
+
+
+def test_deterministic(sv):
+    st, _ = inputs((1, 4, 6000, 128), 9, "bf16")
+    q, k, v = (dev(x, "bf16") for x in st)
+    a = sv.sv_block_causal_attn(q, k, v, 1500, eps=EPS)
+    b = sv.sv_block_causal_attn(q, k, v, 1500, eps=EPS)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_gpu_validation_launches_nothing(sv):
+    import ctypes
+    lib = sv.load()
+    q = torch.zeros(1, 1, 256, 128, dtype=torch.bfloat16, device="cuda")
+    ws = sv.make_workspace(sv.SV_OP_LINATTN_FWD, q)
+    p = ctypes.c_void_p
+    st = lib.sv_linattn_fwd(p(q.data_ptr() + 2), p(q.data_ptr()), p(q.data_ptr()), p(q.data_ptr()), 1, 1, 256, 128,
+                            0, 1e-6, ws.ptr, ws.nbytes, None)
+    assert st == 1 and b"aligned" in lib.sv_last_error()
+    st = lib.sv_linattn_fwd(p(q.data_ptr()), p(q.data_ptr()), p(q.data_ptr()), p(q.data_ptr()), 1, 1, 256, 128,
+                            0, 1e-6, ws.ptr, 1024, None)
+    assert st == 1 and b"workspace" in lib.sv_last_error()
+    assert lib.sv_workspace_bytes(0, 1, 1, 256, 128, 256, 0) == ws.nbytes
+    assert ws.status() == 0
+
+
+# --------------------------------------------------------------------------------------------
+# config 1: 480p bidirectional [2, 20, 8190, 112], full comparison
+# --------------------------------------------------------------------------------------------
+def test_c1_480p_bidirectional_full(sv):
+    st, (q, k, v) = inputs((2, 20, 8190, 112), 0, "bf16")
+    qd, kd, vd = (dev(x, "bf16") for x in st)
+    o = sv.sv_linattn_fwd(qd, kd, vd, eps=EPS)
+    torch.cuda.synchronize()
+    err = oracle.max_rel_err(host(o), oracle.linattn_fwd(q, k, v, EPS))
+    assert err < TOL["bf16"], err
+
+
+# --------------------------------------------------------------------------------------------
+# config 2: 720p block-causal prefill at full size (the bench launch), sampled heads and rows
+# --------------------------------------------------------------------------------------------
+def _sampled_check(o_dev, q, k, v, L, heads, nrows, seed, S_out=None, z_out=None):
+    rng = np.random.default_rng(seed)
+    N = q.shape[2]
+    for (b, h) in heads:
+        S, z = oracle.block_states(k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], L)
+        P, zP = oracle.prefix_states(S, z)
+        rows = np.unique(np.concatenate([rng.integers(0, N, nrows), np.arange(0, N, L), np.arange(L - 1, N, L), [N - 1]]))
+        rows = rows[rows < N]
+        blk = rows // L
+        ref = oracle.rows_from_states(q[b, h, rows], P[0, 0, blk], zP[0, 0, blk], EPS)
+        got = o_dev[b, h, torch.from_numpy(rows).cuda()].float().cpu().numpy()
+        err = oracle.max_rel_err(got, ref)
+        assert err < TOL["bf16"], (b, h, err)
+        if S_out is not None:
+            assert oracle.max_rel_err(host(S_out[b, h]), P[0, 0, -1]) < TOL_CACHE
+            assert oracle.max_rel_err(host(z_out[b, h]), zP[0, 0, -1]) < TOL_CACHE
+
+
+def test_c2_720p_prefill_full_size_sampled(sv):
+    B, H, N, D, L = 1, 20, 55200, 128, 2760
+    st, (q, k, v) = inputs((B, H, N, D), 0, "bf16")
+    qd, kd, vd = (dev(x, "bf16") for x in st)
+    S_out = torch.zeros(B, H, D, D, device="cuda")
+    z_out = torch.zeros(B, H, D, device="cuda")
+    o = sv.sv_block_causal_attn(qd, kd, vd, L, eps=EPS, S_out=S_out, z_out=z_out)
+    torch.cuda.synchronize()
+    _sampled_check(o, q, k, v, L, [(0, 0), (0, 9), (0, 19)], 400, 0, S_out, z_out)
+
+
+# --------------------------------------------------------------------------------------------
+# config 3: 60 streaming blocks of [1, 20, 2760, 128] through the fp32 cache
+# --------------------------------------------------------------------------------------------
+def test_c3_streaming_60_blocks_constant_cache(sv):
+    B, H, D, Lb, nb = 1, 20, 128, 2760, 60
+    S = torch.zeros(B, H, D, D, device="cuda")
+    z = torch.zeros(B, H, D, device="cuda")
+    cache_bytes = S.numel() * 4 + z.numel() * 4
+    assert cache_bytes == B * H * D * (D + 1) * 4 == 1_320_960
+    heads = [0, 13]
+    S_ref = np.zeros((1, len(heads), D, D))
+    z_ref = np.zeros((1, len(heads), D))
+    ws = None
+    mem = None
+    for c in range(nb):
+        st, (q, k, v) = inputs((B, H, Lb, D), c, "bf16")   # block c is drawn with seed c
+        qd, kd, vd = (dev(x, "bf16") for x in st)
+        if ws is None:
+            ws = sv.make_workspace(sv.SV_OP_CACHE_STEP, qd)
+        o = sv.sv_cache_step(qd, kd, vd, S, z, commit=True, eps=EPS, ws=ws)
+        torch.cuda.synchronize()
+        o_ref, S_ref, z_ref = oracle.cache_step(q[:, heads], k[:, heads], v[:, heads], S_ref, z_ref, EPS)
+        if c in (0, 1, 29, 59):
+            assert oracle.max_rel_err(host(o[:, heads]), o_ref) < TOL["bf16"], c
+        del qd, kd, vd, o
+        if c == 1:
+            mem = torch.cuda.memory_allocated()
+        elif c > 1:
+            assert torch.cuda.memory_allocated() == mem  # nothing grows with the number of blocks
+        assert S.shape == (B, H, D, D) and z.shape == (B, H, D)
+    assert oracle.max_rel_err(host(S[:, heads]), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z[:, heads]), z_ref) < TOL_CACHE
+    assert ws.status() == 0
+
+
+# --------------------------------------------------------------------------------------------
+# config 4: SANA-Video 2.0-shaped layers [2, 20, 10120, 128], bidirectional, seed = layer,
+# back to back on one stream (first and last of the 24 layers checked)
+# --------------------------------------------------------------------------------------------
+def test_c4_layers_back_to_back(sv):
+    shape = (2, 20, 10120, 128)
+    layers = [0, 23]
+    data = {l: inputs(shape, l, "bf16") for l in layers}
+    devs = {l: tuple(dev(x, "bf16") for x in data[l][0]) for l in layers}
+    ws = sv.make_workspace(sv.SV_OP_LINATTN_FWD, devs[0][0])
+    outs = {l: sv.sv_linattn_fwd(*devs[l], eps=EPS, ws=ws) for l in layers}
+    torch.cuda.synchronize()
+    for l in layers:
+        q, k, v = data[l][1]
+        for (b, h) in [(0, 0), (1, 19), (1, 7)]:
+            ref = oracle.linattn_fwd(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], EPS)
+            err = oracle.max_rel_err(host(outs[l][b:b + 1, h:h + 1]), ref)
+            assert err < TOL["bf16"], (l, b, h, err)
+    assert ws.status() == 0

@@ -1,0 +1,73 @@
+"""Host-side checks that need no GPU: the geometry shared by the kernels, the library's exported
+symbols, and argument validation that must reject bad calls before any CUDA call."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_geometry_invariants(tmp_path):
+    exe = tmp_path / "geometry_check"
+    subprocess.check_call(["g++", "-O1", "-std=c++17", os.path.join(ROOT, "tests", "geometry_check.cpp"), "-o", str(exe)])
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_causal_linear_relu_b200 import build
+    build.build()
+    import block_causal_linear_relu_b200 as sv
+    return sv.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "svlinattn.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*]+\s+\*?(sv_\w+)\s*\(", text, re.M)))
+
+
+def test_header_and_binding_agree():
+    import block_causal_linear_relu_b200 as sv
+    assert _declared() == sorted(sv.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    nm = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (sv_\w+)", nm))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    assert lib.sv_version() == 100
+    assert lib.sv_last_error() is not None
+
+
+def test_validation_rejects_before_any_launch(lib):
+    # null pointers and bad sizes are refused on the host with no CUDA call (no GPU here)
+    vp = ctypes.c_void_p
+    f = lib.sv_linattn_fwd
+    fake = vp(256 * 1024)
+    assert f(None, fake, fake, fake, 1, 1, 128, 128, 0, 1e-6, fake, 1 << 30, None) == 1
+    assert b"q is NULL" in lib.sv_last_error()
+    assert f(fake, fake, fake, fake, 1, 1, 0, 128, 0, 1e-6, fake, 1 << 30, None) == 1      # N = 0
+    assert f(fake, fake, fake, fake, 1, 1, 128, 100, 0, 1e-6, fake, 1 << 30, None) == 2    # bf16 D=100
+    assert f(fake, fake, fake, fake, 1, 1, 128, 32, 0, 1e-6, fake, 1 << 30, None) == 2     # bf16 D=32
+    assert f(fake, fake, fake, fake, 1, 1, 128, 129, 1, 1e-6, fake, 1 << 30, None) == 2    # f32 D>128
+    assert f(fake, fake, fake, fake, 1, 1, 128, 128, 7, 1e-6, fake, 1 << 30, None) == 2    # dtype
+    assert f(fake, vp(256 * 1024 + 2), fake, fake, 1, 1, 128, 128, 0, 1e-6, fake, 1 << 30, None) == 1  # misaligned
+    assert b"16-byte aligned" in lib.sv_last_error()
+    bc = lib.sv_block_causal_attn
+    assert bc(fake, fake, fake, fake, 1, 1, 128, 128, 0, 0, 1e-6, None, None, None, None, fake, 1 << 30, None) == 1
+    assert b"block_len" in lib.sv_last_error()
+    assert bc(fake, fake, fake, fake, 1, 1, 128, 128, 64, 0, float("nan"), None, None, None, None, fake, 1 << 30, None) == 1
+    assert bc(fake, fake, fake, fake, 1, 1, 128, 128, 64, 0, 1e-6, vp(256 * 1024 + 1), None, None, None, fake, 1 << 30, None) == 1
+    cs = lib.sv_cache_step
+    assert cs(fake, fake, fake, fake, 1, 1, 128, 128, 0, 1e-6, None, fake, 1, fake, 1 << 30, None) == 1
+    assert b"S is NULL" in lib.sv_last_error()
+    su = lib.sv_block_state_update
+    assert su(fake, fake, 1, 1, 128, 128, 0, fake, None, fake, 1 << 30, None) == 1
+    assert lib.sv_workspace_init(None, 0, None) == 1
