@@ -123,6 +123,7 @@ sv_status make_block_maps(sv::BlockMaps& bm, const void* x, const Geom& g, uint3
 
 // ---- workspace layout ----
 struct WsLayout {
+  size_t segcta = 0;    // offset of the per-segment (first CTA, last CTA) table
   size_t partials = 0;  // offset of the fp32 partial slots
   size_t ptiles = 0;    // offset of the prefix tiles (bf16 B operands or fp32 prefixes)
   size_t total = 0;
@@ -133,6 +134,8 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 WsLayout ws_layout(const Geom& g, sv_dtype dt, bool need_prefix) {
   WsLayout w;
   size_t off = sv::kHeaderBytes;
+  w.segcta = off;
+  off += align256(static_cast<size_t>(g.nseg) * sizeof(int2));
   w.partials = off;
   off += align256(static_cast<size_t>(g.nslots) * sv::kPartBytes);
   w.ptiles = off;
@@ -215,6 +218,7 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
   float* partials = reinterpret_cast<float*>(wsb + lay.partials);
+  int2* segcta = reinterpret_cast<int2*>(wsb + lay.segcta);
   void* pre = wsb + lay.ptiles;
   cudaError_t e;
   if (dt == SV_BF16) {
@@ -224,10 +228,10 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
     SV_TRY(make_block_maps(mq, q, g, sv::kTile));
     SV_TRY(make_block_maps(mo, o, g, 32));
     prof_mark(0, stream);
-    e = sv::launch_state_bf16(mk, mv, g, partials, status, stream);
+    e = sv::launch_state_bf16(mk, mv, g, partials, segcta, status, stream);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
     prof_mark(1, stream);
-    e = sv::launch_scan(partials, g, S_in, z_in, S_out, z_out, pre, nullptr, stream);
+    e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, pre, nullptr, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     prof_mark(2, stream);
     e = sv::launch_out_bf16(mq, mo, g, pre, eps, status, stream);
@@ -236,11 +240,11 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
   } else {
     float* p32 = static_cast<float*>(pre);
     prof_mark(0, stream);
-    e = sv::launch_state_f32(static_cast<const float*>(k), static_cast<const float*>(v), g, partials, status,
-                             stream);
+    e = sv::launch_state_f32(static_cast<const float*>(k), static_cast<const float*>(v), g, partials, segcta,
+                             status, stream);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
     prof_mark(1, stream);
-    e = sv::launch_scan(partials, g, S_in, z_in, S_out, z_out, nullptr, p32, stream);
+    e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, nullptr, p32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     prof_mark(2, stream);
     e = sv::launch_out_f32(static_cast<const float*>(q), static_cast<float*>(o), g, p32, eps, status, stream);
@@ -332,17 +336,19 @@ sv_status sv_block_state_update(const void* k, const void* v, int B, int H, int 
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
   float* partials = reinterpret_cast<float*>(wsb + lay.partials);
+  int2* segcta = reinterpret_cast<int2*>(wsb + lay.segcta);
   cudaError_t e;
   if (dt == SV_BF16) {
     sv::BlockMaps mk, mv;
     SV_TRY(make_block_maps(mk, k, g, sv::kTile));
     SV_TRY(make_block_maps(mv, v, g, sv::kTile));
-    e = sv::launch_state_bf16(mk, mv, g, partials, status, s);
+    e = sv::launch_state_bf16(mk, mv, g, partials, segcta, status, s);
   } else {
-    e = sv::launch_state_f32(static_cast<const float*>(k), static_cast<const float*>(v), g, partials, status, s);
+    e = sv::launch_state_f32(static_cast<const float*>(k), static_cast<const float*>(v), g, partials, segcta,
+                             status, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
-  e = sv::launch_scan(partials, g, S, z, S, z, nullptr, nullptr, s);
+  e = sv::launch_scan(partials, segcta, g, S, z, S, z, nullptr, nullptr, s);
   if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
   return SV_OK;
 }

@@ -16,23 +16,18 @@ struct BlockMaps {
   CUtensorMap last;
 };
 
-struct Bf16Launch {
-  BlockMaps q, k, v, o;     // q/k/v: 128-row load boxes; o: 32-row store boxes
-  const uint16_t* ptiles;   // workspace: bf16 prefix tiles (nseg x kPTileBytes)
-};
-
 // bf16 path
-cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials,
+cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,
                               uint32_t* status, cudaStream_t st);
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles,
                             float eps, uint32_t* status, cudaStream_t st);
 // fp32 path
-cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, uint32_t* status,
-                             cudaStream_t st);
+cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
+                             uint32_t* status, cudaStream_t st);
 cudaError_t launch_out_f32(const float* q, float* o, const Geom& g, const float* p32, float eps,
                            uint32_t* status, cudaStream_t st);
 // both paths: combine partials, inclusive prefix over blocks, optional final cache
-cudaError_t launch_scan(const float* partials, const Geom& g, const float* S_in, const float* z_in,
+cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
                         float* S_out, float* z_out, void* ptiles_bf16, float* p32, cudaStream_t st);
 
 size_t state_bf16_smem_bytes();

@@ -17,6 +17,8 @@
 // The fp32 I/O path runs the same three steps with SIMT fp32 kernels.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "sv_internal.h"
 #include "sv_ptx.cuh"
 
@@ -70,7 +72,8 @@ constexpr int kSmemBytes = kBarOff + 256 + 1024;
 __global__ void __launch_bounds__(kThreads, 1)
     state_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
                       const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
-                      const Geom geo, float* __restrict__ partials, uint32_t* status) {
+                      const Geom geo, float* __restrict__ partials, int2* __restrict__ segcta,
+                      uint32_t* status) {
   using namespace st;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -133,11 +136,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == kWarpProducer) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const uint32_t tx = two_atoms ? 2u * kKBytes : static_cast<uint32_t>(kKBytes);
+      // K, V may come from the previous kernel in the stream, and the partial slots written below
+      // may still be read by the previous call's scan: nothing is touched before this wait.
+      griddep_wait();
       int k = 0;
       for (long long t = tb; t < te; ++t, ++k) {
         const TileCoord c = tile_coord(t, geo);
@@ -237,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_x1(ta + 128, zr);
       tmem_wait_ld();
       dst[kZRow * kDPad + d] = __uint_as_float(zr);
+      if (warp == 0 && lane == 0) {  // which CTAs hold the first and the last tile of the segment
+        if (t - c.tok0 / kTile >= tb) segcta[c.seg].x = g;
+        if (c.last) segcta[c.seg].y = g;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[a]);
@@ -321,13 +332,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (threadIdx.x == 0) griddep_launch_dependents();
+
   if (warp == kWarpProducer) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const uint32_t tx = two_atoms ? static_cast<uint32_t>(kQBytes) : static_cast<uint32_t>(kAtomBytes);
+      auto load_q = [&](long long t, int s) {
+        const TileCoord c = tile_coord(t, geo);
+        const bool lst = use_last_map(c, geo);
+        const CUtensorMap* mq = lst ? &q_last : &q_main;
+        const int cb = lst ? 0 : c.blk;
+        uint8_t* stg = smem + s * kQBytes;
+        mbar_expect_tx(&qfull[s], tx);
+        tma_load_4d(stg, mq, &qfull[s], 0, c.tok0, cb, c.bh, pol);
+        if (two_atoms) tma_load_4d(stg + kAtomBytes, mq, &qfull[s], 64, c.tok0, cb, c.bh, pol);
+      };
+      // Q was final before the state kernel ran, so the first stages fill while the scan runs;
+      // the prefix tiles are read only after the scan grid has completed.
+      const int pre = static_cast<int>(te - tb < kStages ? te - tb : kStages);
+      for (int i = 0; i < pre; ++i) load_q(tb + i, i);
+      griddep_wait();
       int k = 0, j = 0, prev = -1;
-      bool ok = true;
-      for (long long t = tb; t < te && ok; ++t, ++k) {
+      for (long long t = tb; t < te; ++t, ++k) {
         const TileCoord c = tile_coord(t, geo);
         if (c.seg != prev) {
           const int bb = j & 1;
@@ -338,17 +365,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++j;
           prev = c.seg;
         }
-        const int s = k % kStages;
-        if (!mbar_wait(&qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) break;
-        const bool lst = use_last_map(c, geo);
-        const CUtensorMap* mq = lst ? &q_last : &q_main;
-        const int cb = lst ? 0 : c.blk;
-        uint8_t* stg = smem + s * kQBytes;
-        mbar_expect_tx(&qfull[s], tx);
-        tma_load_4d(stg, mq, &qfull[s], 0, c.tok0, cb, c.bh, pol);
-        if (two_atoms) tma_load_4d(stg + kAtomBytes, mq, &qfull[s], 64, c.tok0, cb, c.bh, pol);
+        if (k >= pre) {
+          const int s = k % kStages;
+          if (!mbar_wait(&qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) break;
+          load_q(t, s);
+        }
       }
-      for (int i = (k > kStages ? k - kStages : 0); i < k; ++i)
+      for (int i = (k > kStages ? k - kStages : 0); i < (k > pre ? k : pre); ++i)
         mbar_wait(&qfull[i % kStages], (i / kStages) & 1, status, 0x1180u);
       for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&bfull[i & 1], (i >> 1) & 1, status, 0x1190u);
     }
@@ -465,67 +488,129 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------------------
 // 2. partial combine + inclusive prefix over blocks (+ incoming cache), both paths
 // ------------------------------------------------------------------------------------------
-// One thread per (bh, row e of the prefix tile, 4 consecutive key features d).
-__global__ void __launch_bounds__(256) scan_kernel(const float* __restrict__ partials, const Geom geo,
-                                                   const float* S_in, const float* z_in, float* S_out,
-                                                   float* z_out, uint8_t* __restrict__ ptiles,
-                                                   float* __restrict__ p32) {
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long total = static_cast<long long>(geo.BH) * kPTileRows * 32;
-  if (idx >= total) return;
-  const int quad = static_cast<int>(idx & 31);
-  const int e = static_cast<int>((idx >> 5) % kPTileRows);
-  const int bh = static_cast<int>((idx >> 5) / kPTileRows);
+// CTA (bh, row e of the prefix tile): e < 128 are S^T rows (value feature e), e = 128 is z,
+// e = 129..143 are the zero rows of the bf16 B operand. Lane q owns key features 4q..4q+3;
+// warp j owns blocks [j*nblk/ng, (j+1)*nblk/ng) (at most kScanReg of them when nblk <= 128),
+// so every partial load is independent; the running prefix crosses warps through shared memory.
+constexpr int kScanReg = 4;
+constexpr int kScanMaxWarps = 32;
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+// Sum of the partial slots g + seg of the CTAs g0..g1 that covered segment `seg` (the state kernel
+// records g0/g1 per segment while it flushes).
+__device__ __forceinline__ float4 block_sum(const float* __restrict__ partials, const int2* __restrict__ segcta,
+                                            int seg, int e, int d0) {
+  const int2 r = segcta[seg];
+  const int g0 = r.x, g1 = r.y;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int gg = g0; gg <= g1; ++gg)
+    acc = f4add(acc, *reinterpret_cast<const float4*>(
+                         partials + (static_cast<size_t>(gg + seg) * kPartRows + e) * kDPad + d0));
+  return acc;
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ partials,
+                                                    const int2* __restrict__ segcta, const Geom geo,
+                                                    const float* S_in, const float* z_in, float* S_out,
+                                                    float* z_out, uint8_t* __restrict__ ptiles,
+                                                    float* __restrict__ p32) {
+  griddep_wait();  // partials come from the state kernel; prefix tiles may still be read before it
+  griddep_launch_dependents();
+  extern __shared__ float4 s_scan[];   // [ng][32] warp totals, then [32] incoming cache
+  float4* s_base = s_scan + (blockDim.x >> 5) * 32;
+  const int bh = blockIdx.x;
+  const int e = blockIdx.y;
+  const int q = threadIdx.x & 31;
+  const int j = threadIdx.x >> 5;
+  const int ng = blockDim.x >> 5;
+  const int nblk = geo.nblk;
   const int D = geo.D;
-  const int d0 = quad * 4;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (S_in != nullptr && e < D) {
+  const int d0 = q * 4;
+  const int c0 = static_cast<int>(static_cast<long long>(j) * nblk / ng);
+  const int c1 = static_cast<int>(static_cast<long long>(j + 1) * nblk / ng);
+  const int cnt = c1 - c0;
+  const bool live = e < kPartRows;
+  const int seg0 = bh * nblk;
+
+  // pass 1: this warp's block sums (kept in registers) and their total
+  float4 sums[kScanReg];
+  float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (d0 + u < D) acc[u] = S_in[(static_cast<size_t>(bh) * D + d0 + u) * D + e];
-  }
-  if (z_in != nullptr && e == kZRow) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (d0 + u < D) acc[u] = z_in[static_cast<size_t>(bh) * D + d0 + u];
-  }
-  for (int b = 0; b < geo.nblk; ++b) {
-    const int seg = bh * geo.nblk + b;
-    if (e < kPartRows) {
-      const long long first = seg_first_tile(seg, geo);
-      const int g0 = cta_of_tile(first, geo);
-      const int g1 = cta_of_tile(first + seg_ntiles(seg, geo) - 1, geo);
-      for (int gg = g0; gg <= g1; ++gg) {
-        const float4 p = *reinterpret_cast<const float4*>(
-            partials + (static_cast<size_t>(gg + seg) * kPartRows + e) * kDPad + d0);
-        acc[0] += p.x;
-        acc[1] += p.y;
-        acc[2] += p.z;
-        acc[3] += p.w;
-      }
+  for (int i = 0; i < kScanReg; ++i) {
+    sums[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live && i < cnt) {
+      sums[i] = block_sum(partials, segcta, seg0 + c0 + i, e, d0);
+      tot = f4add(tot, sums[i]);
     }
+  }
+  for (int i = kScanReg; i < cnt; ++i)
+    if (live) tot = f4add(tot, block_sum(partials, segcta, seg0 + c0 + i, e, d0));
+
+  // incoming cache (S_in row e of S^T, or z_in for the z row)
+  float base[4] = {0.f, 0.f, 0.f, 0.f};
+  if (j == 0) {
+    if (S_in != nullptr && e < D) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (d0 + u < D) base[u] = S_in[(static_cast<size_t>(bh) * D + d0 + u) * D + e];
+    }
+    if (z_in != nullptr && e == kZRow) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (d0 + u < D) base[u] = z_in[static_cast<size_t>(bh) * D + d0 + u];
+    }
+  }
+  float4 run = make_float4(base[0], base[1], base[2], base[3]);
+  if (ng > 1) {
+    s_scan[j * 32 + q] = tot;
+    if (j == 0) s_base[q] = run;
+    __syncthreads();
+    run = s_base[q];
+    for (int jj = 0; jj < j; ++jj) run = f4add(run, s_scan[jj * 32 + q]);
+  }
+
+  // pass 2: running prefix, one prefix tile row chunk per block
+  auto emit = [&](int c, const float4& r) {
+    const int seg = seg0 + c;
     if (ptiles != nullptr) {
       uint2 w;
-      w.x = pack_bf16x2(acc[0], acc[1]);
-      w.y = pack_bf16x2(acc[2], acc[3]);
+      w.x = pack_bf16x2(r.x, r.y);
+      w.y = pack_bf16x2(r.z, r.w);
       const size_t off = static_cast<size_t>(seg) * kPTileBytes + (d0 >> 6) * (kPTileRows * 128) + e * 128 +
                          ((((d0 & 63) >> 3) ^ (e & 7)) << 4) + (d0 & 7) * 2;
       *reinterpret_cast<uint2*>(ptiles + off) = w;
     }
-    if (p32 != nullptr && e < kPartRows) {
-      *reinterpret_cast<float4*>(p32 + (static_cast<size_t>(seg) * kPartRows + e) * kDPad + d0) =
-          make_float4(acc[0], acc[1], acc[2], acc[3]);
+    if (p32 != nullptr && live)
+      *reinterpret_cast<float4*>(p32 + (static_cast<size_t>(seg) * kPartRows + e) * kDPad + d0) = r;
+  };
+#pragma unroll
+  for (int i = 0; i < kScanReg; ++i) {
+    if (i < cnt) {
+      run = f4add(run, sums[i]);
+      emit(c0 + i, run);
     }
   }
-  if (S_out != nullptr && e < D) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (d0 + u < D) S_out[(static_cast<size_t>(bh) * D + d0 + u) * D + e] = acc[u];
+  for (int i = kScanReg; i < cnt; ++i) {
+    if (live) run = f4add(run, block_sum(partials, segcta, seg0 + c0 + i, e, d0));
+    emit(c0 + i, run);
   }
-  if (z_out != nullptr && e == kZRow) {
+
+  // final cache: the warp holding the last block
+  if (c1 == nblk && cnt > 0) {
+    const float r[4] = {run.x, run.y, run.z, run.w};
+    if (S_out != nullptr && e < D) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (d0 + u < D) z_out[static_cast<size_t>(bh) * D + d0 + u] = acc[u];
+      for (int u = 0; u < 4; ++u)
+        if (d0 + u < D) S_out[(static_cast<size_t>(bh) * D + d0 + u) * D + e] = r[u];
+    }
+    if (z_out != nullptr && e == kZRow) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (d0 + u < D) z_out[static_cast<size_t>(bh) * D + d0 + u] = r[u];
+    }
   }
 }
 
@@ -540,7 +625,7 @@ constexpr int kOutF32Smem = kDPad * kPartRows * 4 + kTile * kDPad * 4;  // prefi
 
 __global__ void __launch_bounds__(kF32Threads, 1)
     state_f32_kernel(const float* __restrict__ k, const float* __restrict__ v, const Geom geo,
-                     float* __restrict__ partials) {
+                     float* __restrict__ partials, int2* __restrict__ segcta) {
   extern __shared__ float fsm[];
   float* Ks = fsm;
   float* Vs = fsm + kTile * kDPad;
@@ -586,6 +671,10 @@ __global__ void __launch_bounds__(kF32Threads, 1)
       }
       if (eh == 0) dst[kZRow * kDPad + d] = (d < D) ? zacc : 0.f;
       zacc = 0.f;
+      if (threadIdx.x == 0) {
+        if (t - c.tok0 / kTile >= tb) segcta[c.seg].x = g;
+        if (c.last) segcta[c.seg].y = g;
+      }
     }
   }
 }
@@ -641,6 +730,25 @@ __global__ void __launch_bounds__(kF32Threads, 1)
 // ------------------------------------------------------------------------------------------
 // launchers
 // ------------------------------------------------------------------------------------------
+// Every launch allows programmatic dependent launch: a kernel may be scheduled while the previous
+// one in the stream drains, and each kernel waits (griddepcontrol.wait) before touching memory
+// that the previous kernels write or still read.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 size_t state_bf16_smem_bytes() { return st::kSmemBytes; }
 size_t out_bf16_smem_bytes() { return ot::kSmemBytes; }
 size_t state_f32_smem_bytes() { return kStateF32Smem; }
@@ -657,31 +765,31 @@ cudaError_t set_kernel_attributes() {
   return cudaFuncSetAttribute(out_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutF32Smem);
 }
 
-cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials,
+cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,
                               uint32_t* status, cudaStream_t s) {
-  state_bf16_kernel<<<g.G, kThreads, st::kSmemBytes, s>>>(k.main, k.last, v.main, v.last, g, partials, status);
-  return cudaGetLastError();
+  return launch_pdl(state_bf16_kernel, dim3(g.G), dim3(kThreads), st::kSmemBytes, s, k.main, k.last, v.main, v.last,
+                    g, partials, segcta, status);
 }
 
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles, float eps,
                             uint32_t* status, cudaStream_t s) {
-  out_bf16_kernel<<<g.G, kThreads, ot::kSmemBytes, s>>>(q.main, q.last, o.main, o.last, g,
-                                                        static_cast<const uint8_t*>(ptiles), eps, status);
-  return cudaGetLastError();
+  return launch_pdl(out_bf16_kernel, dim3(g.G), dim3(kThreads), ot::kSmemBytes, s, q.main, q.last, o.main, o.last,
+                    g, static_cast<const uint8_t*>(ptiles), eps, status);
 }
 
-cudaError_t launch_scan(const float* partials, const Geom& g, const float* S_in, const float* z_in, float* S_out,
+cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in, float* S_out,
                         float* z_out, void* ptiles_bf16, float* p32, cudaStream_t s) {
-  const long long total = static_cast<long long>(g.BH) * kPTileRows * 32;
-  const int blocks = static_cast<int>((total + 255) / 256);
-  scan_kernel<<<blocks, 256, 0, s>>>(partials, g, S_in, z_in, S_out, z_out, static_cast<uint8_t*>(ptiles_bf16),
-                                     p32);
-  return cudaGetLastError();
+  int ng = (g.nblk + kScanReg - 1) / kScanReg;
+  if (ng > kScanMaxWarps) ng = kScanMaxWarps;
+  if (ng < 1) ng = 1;
+  return launch_pdl(scan_kernel, dim3(g.BH, kPTileRows), dim3(32 * ng), (ng + 1) * 32 * sizeof(float4), s,
+                    partials, segcta, g, S_in, z_in, S_out,
+                    z_out, static_cast<uint8_t*>(ptiles_bf16), p32);
 }
 
-cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, uint32_t*,
-                             cudaStream_t s) {
-  state_f32_kernel<<<g.G, kF32Threads, kStateF32Smem, s>>>(k, v, g, partials);
+cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
+                             uint32_t*, cudaStream_t s) {
+  state_f32_kernel<<<g.G, kF32Threads, kStateF32Smem, s>>>(k, v, g, partials, segcta);
   return cudaGetLastError();
 }
 
