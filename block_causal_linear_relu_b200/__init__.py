@@ -21,6 +21,7 @@ from ._native import (  # noqa: F401
     sv_block_causal_attn,
     sv_block_state_update,
     sv_cache_step,
+    sv_cache_step_noalloc,
     sv_linattn_fwd,
     sv_profile_events,
     workspace_bytes,

@@ -25,8 +25,8 @@ SV_OP_LINATTN_FWD, SV_OP_BLOCK_STATE_UPDATE, SV_OP_BLOCK_CAUSAL_ATTN, SV_OP_CACH
 #: every symbol include/svlinattn.h declares
 EXPORTS = (
     "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_linattn_fwd",
-    "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_profile_events", "sv_last_error",
-    "sv_version",
+    "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_cache_step_noalloc",
+    "sv_profile_events", "sv_last_error", "sv_version",
 )
 
 
@@ -64,6 +64,8 @@ def load() -> ctypes.CDLL:
         lib.sv_block_causal_attn.restype = i
         lib.sv_cache_step.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, vp, vp, i, vp, sz, vp]
         lib.sv_cache_step.restype = i
+        lib.sv_cache_step_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, vp, vp, i, vp]
+        lib.sv_cache_step_noalloc.restype = i
         lib.sv_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
         lib.sv_profile_events.restype = i
         lib.sv_last_error.argtypes = []
@@ -187,6 +189,18 @@ def sv_cache_step(q, k, v, S, z, commit: bool = True, o=None, eps: float = 1e-6,
     ws = _ws(ws, SV_OP_CACHE_STEP, q, None, stream)
     _check(load().sv_cache_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, _ptr(S), _ptr(z),
                                 1 if commit else 0, ws.ptr, ws.nbytes, _stream(stream)))
+    return o
+
+
+def sv_cache_step_noalloc(q, k, v, S, z, commit: bool = True, o=None, eps: float = 1e-6, stream=None):
+    """sv_cache_step with the library's static scratch instead of a workspace (see the header)."""
+    B, H, N, D = _qkv(q, k, v)
+    o = torch.empty_like(q) if o is None else o
+    _qkv(q, o)
+    if S.dtype != torch.float32 or z.dtype != torch.float32 or tuple(S.shape) != (B, H, D, D) or tuple(z.shape) != (B, H, D):
+        raise ValueError("cache must be float32 S [B,H,D,D] and z [B,H,D]")
+    _check(load().sv_cache_step_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, _ptr(S),
+                                        _ptr(z), 1 if commit else 0, _stream(stream)))
     return o
 
 

@@ -256,6 +256,13 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
 
 }  // namespace
 
+namespace sv {
+sv_status set_last_error(sv_status status, const char* msg) {
+  g_last_error = msg;
+  return status;
+}
+}  // namespace sv
+
 extern "C" {
 
 size_t sv_workspace_bytes(sv_op op, int B, int H, int N, int D, int block_len, sv_dtype dt) {

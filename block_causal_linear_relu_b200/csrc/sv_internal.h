@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/svlinattn.h"
 #include "sv_geometry.h"
 
 namespace sv {
@@ -29,6 +30,9 @@ cudaError_t launch_out_f32(const float* q, float* o, const Geom& g, const float*
 // both paths: combine partials, inclusive prefix over blocks, optional final cache
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
                         float* S_out, float* z_out, void* ptiles_bf16, float* p32, cudaStream_t st);
+
+// Records `msg` as the calling thread's sv_last_error() text and returns `status`.
+sv_status set_last_error(sv_status status, const char* msg);
 
 size_t state_bf16_smem_bytes();
 size_t out_bf16_smem_bytes();

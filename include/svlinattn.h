@@ -110,6 +110,23 @@ sv_status sv_cache_step(const void* q, const void* k, const void* v, void* o, in
                         sv_dtype dt, float eps, float* S, float* z, int commit, void* ws, size_t ws_bytes,
                         sv_stream_t stream);
 
+/* sv_cache_step without a workspace argument, for callers that cannot allocate device memory:
+ * an operator called from a host framework that owns all memory, a real-time block loop that must
+ * not call cudaMalloc (it synchronises the device), or code being recorded into a CUDA graph,
+ * where allocation is not allowed while recording. The paper has no counterpart; this is a
+ * deployment convenience of this library.
+ * Scratch comes from one static device array of 16 MiB compiled into the library (held on every
+ * device that loads the library until the process exits). Arguments and results are those of
+ * sv_cache_step. A call that needs more scratch than 16 MiB (see sv_workspace_bytes with
+ * SV_OP_CACHE_STEP: about 66 KB per (batch, head) pair plus 66 KB per streaming multiprocessor,
+ * so the 720p streaming block [1, 20, 2760, 128] needs about 12 MB and B * H above ~100 does not
+ * fit) is refused with SV_ERR_INVALID_ARG before any launch. All calls on a device share the array: calls that may
+ * overlap on the GPU race. The first call on a device looks up the array's device address; make
+ * it before any stream capture. Device-side wait timeouts are not reported through this entry
+ * point (use sv_cache_step with a workspace and sv_device_status for that). */
+sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                                sv_dtype dt, float eps, float* S, float* z, int commit, sv_stream_t stream);
+
 /* Optional timing hook for benchmarks. With events != NULL (n == 4 cudaEvent_t handles owned by
  * the caller), the calling thread's following forward calls (sv_linattn_fwd, sv_block_causal_attn,
  * sv_cache_step) record events[0] before the state-reduction kernel, events[1] after it,
