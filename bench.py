@@ -341,6 +341,75 @@ def run_ours(args, rank: int, world: int):
     return 0
 
 
+EXTRA_WORKLOADS = {
+    # name: (description, B, H, N, D, block_len, kind, repeats)
+    "480p_bidir": ("480p bidirectional Linear DiT attention: B=2 H=20 N=8190 (21x15x26) D=112", 2, 20, 8190, 112,
+                   8190, "fwd", 1),
+    "720p_stream": ("autoregressive cache streaming: 60 blocks of B=1 H=20 N=2760 D=128 through the fp32 cache "
+                    "(S [1,20,128,128], z [1,20,128]), one sv_cache_step per block", 1, 20, 2760, 128, 2760,
+                    "stream", 60),
+    "sv2_stack": ("SANA-Video 2.0-shaped stack: 24 bidirectional layers of B=2 H=20 N=10120 D=128, fresh inputs "
+                  "per layer, back to back on one stream", 2, 20, 10120, 128, 10120, "fwd", 24),
+}
+
+
+def run_extra(args, name):
+    """Timing of the other configurations (one JSON line; not the default bench line). Inputs come
+    from torch's seeded CUDA generator (seed 0), distinct per layer / per block."""
+    import torch
+
+    import block_causal_linear_relu_b200 as sv
+
+    desc, b, h, n, d, blen, kind, reps = EXTRA_WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sv.load()
+    hbm_gbs, _, _, _ = peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    sets = [tuple(torch.randn(b, h, n, d, device=dev, generator=gen).to(torch.bfloat16) for _ in range(3))
+            for _ in range(reps)]
+    outs = [torch.empty_like(x[0]) for x in sets]
+    S = torch.zeros(b, h, d, d, device=dev)
+    z = torch.zeros(b, h, d, device=dev)
+    op = sv.SV_OP_CACHE_STEP if kind == "stream" else sv.SV_OP_LINATTN_FWD
+    ws = sv.make_workspace(op, sets[0][0])
+    stream = torch.cuda.current_stream()
+
+    def one(i):
+        q, k, v = sets[i]
+        if kind == "stream":
+            sv.sv_cache_step(q, k, v, S, z, commit=True, o=outs[i], ws=ws, stream=stream)
+        else:
+            sv.sv_linattn_fwd(q, k, v, o=outs[i], ws=ws, stream=stream)
+
+    for i in range(min(reps, 3)):
+        one(i)
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(max(1, args.steps // reps)):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        evs[0].record(stream)
+        for i in range(reps):
+            one(i)
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+        per += [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
+    if ws.status() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout")
+    per_ms = np.array(per)
+    tokheads = b * h * n
+    ms = float(per_ms.mean())
+    step_bytes = tokheads * 4 * d * 2
+    line = {"metric": METRIC, "value": tokheads / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "workload": name,
+            "config": {"workload": desc}, "calls_timed": len(per), "ms_per_call_mean": ms,
+            "ms_per_call_median": float(np.median(per_ms)), "ms_per_call_p90": float(np.percentile(per_ms, 90)),
+            "hbm_gbs_alg": step_bytes / (ms / 1e3) / 1e9, "hbm_frac": step_bytes / (ms / 1e3) / 1e9 / hbm_gbs,
+            "dtype": "bf16", "data": "synthetic (torch CUDA generator, seed 0)", "impl": "ours"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -351,6 +420,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["720p_prefill"] + sorted(EXTRA_WORKLOADS), default="720p_prefill",
+                    help="the bench line is 720p_prefill; the others print an informational timing line")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (profiling captures of a smaller case only; not a bench line)")
     args = ap.parse_args()
@@ -365,6 +436,8 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload != "720p_prefill":
+        return run_extra(args, args.workload)
     if world > 1:
         import datetime
 

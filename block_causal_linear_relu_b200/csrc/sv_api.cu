@@ -123,6 +123,7 @@ sv_status make_block_maps(sv::BlockMaps& bm, const void* x, const Geom& g, uint3
 
 // ---- workspace layout ----
 struct WsLayout {
+  size_t flags = 0;     // offset of the per-slot ready / combined flags (single-launch path)
   size_t segcta = 0;    // offset of the per-segment (first CTA, last CTA) table
   size_t partials = 0;  // offset of the fp32 partial slots
   size_t ptiles = 0;    // offset of the prefix tiles (bf16 B operands or fp32 prefixes)
@@ -134,6 +135,8 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 WsLayout ws_layout(const Geom& g, sv_dtype dt, bool need_prefix) {
   WsLayout w;
   size_t off = sv::kHeaderBytes;
+  w.flags = off;
+  off += align256(static_cast<size_t>(g.nslots) * 2 * sizeof(uint64_t));  // ready + combined per slot
   w.segcta = off;
   off += align256(static_cast<size_t>(g.nseg) * sizeof(int2));
   w.partials = off;
@@ -219,6 +222,7 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
   uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
   float* partials = reinterpret_cast<float*>(wsb + lay.partials);
   int2* segcta = reinterpret_cast<int2*>(wsb + lay.segcta);
+  uint64_t* flags = reinterpret_cast<uint64_t*>(wsb + lay.flags);
   void* pre = wsb + lay.ptiles;
   cudaError_t e;
   if (dt == SV_BF16) {
@@ -227,6 +231,16 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
     SV_TRY(make_block_maps(mv, v, g, sv::kTile));
     SV_TRY(make_block_maps(mq, q, g, sv::kTile));
     SV_TRY(make_block_maps(mo, o, g, 32));
+    if (g.nblk == 1) {  // one block: a single fused launch
+      prof_mark(0, stream);
+      e = sv::launch_fused_bf16(mk, mv, mq, mo, g, partials, segcta, flags, pre, S_in, z_in, S_out, z_out, eps,
+                                status, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
+      prof_mark(1, stream);
+      prof_mark(2, stream);
+      prof_mark(3, stream);
+      return SV_OK;
+    }
     prof_mark(0, stream);
     e = sv::launch_state_bf16(mk, mv, g, partials, segcta, status, stream);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
@@ -282,8 +296,9 @@ size_t sv_workspace_bytes(sv_op op, int B, int H, int N, int D, int block_len, s
 sv_status sv_workspace_init(void* ws, size_t ws_bytes, sv_stream_t stream) {
   if (ws == nullptr || ws_bytes < static_cast<size_t>(sv::kHeaderBytes))
     return fail(SV_ERR_INVALID_ARG, "workspace is NULL or smaller than %d bytes", sv::kHeaderBytes);
-  cudaError_t e = cudaMemsetAsync(ws, 0, sv::kHeaderBytes, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  // all of it: the status word, the launch sequence number and the inter-CTA flags start at zero
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
   return SV_OK;
 }
 

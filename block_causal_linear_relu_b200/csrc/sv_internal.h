@@ -22,6 +22,11 @@ cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom
                               uint32_t* status, cudaStream_t st);
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles,
                             float eps, uint32_t* status, cudaStream_t st);
+// bf16, whole sequence in one block: state -> combine -> output in one cooperative launch
+cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
+                              const Geom& g, float* partials, int2* segcta, uint64_t* flags, void* ptiles,
+                              const float* S_in, const float* z_in, float* S_out, float* z_out, float eps,
+                              uint32_t* status, cudaStream_t st);
 // fp32 path
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
                              uint32_t* status, cudaStream_t st);

@@ -58,203 +58,496 @@ __device__ __forceinline__ bool use_last_map(const TileCoord& c, const Geom& g) 
 }
 
 // ------------------------------------------------------------------------------------------
-// 1. block-state reduction (bf16 in, fp32 TMEM accumulation)
+// Pipeline roles. Each persistent kernel runs one CTA per SM with ten warps: warps 0-3 drain the
+// TMEM accumulator (epilogue), warps 4-7 apply ReLU in shared memory, one thread of warp 8 issues
+// TMA copies, one thread of warp 9 issues tcgen05.mma. The roles below are shared by the stand-alone
+// kernels and by the fused single-launch kernel.
 // ------------------------------------------------------------------------------------------
+struct Maps4 {
+  const CUtensorMap* a_main;
+  const CUtensorMap* a_last;
+  const CUtensorMap* b_main;
+  const CUtensorMap* b_last;
+};
+
+// generic-proxy writes to global memory (other CTAs) -> visible to this thread's async-proxy copies
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---- flags between CTAs of the single-launch kernel (release / acquire at GPU scope) ----
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+// Waits (bounded) until flags[i] == tag for every i in [i0, i1]; one thread. Up to eight flags are
+// read per round trip; the fence after the last one orders everything the flag writers released.
+__device__ bool wait_flags(const uint64_t* flags, int i0, int i1, uint64_t tag, uint32_t* status, uint32_t where) {
+  const uint64_t t0 = globaltimer_ns();
+  int i = i0;
+  while (i <= i1) {
+    const int n = (i1 - i + 1) < 8 ? (i1 - i + 1) : 8;
+    uint64_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (u < n) v[u] = ld_relaxed_u64(flags + i + u);
+    int ready = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (u < n && ready == u && v[u] == tag) ++ready;
+    i += ready;
+    if (ready < n) {
+      if (*reinterpret_cast<volatile uint32_t*>(status) != 0u) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kDevTimeout | where);
+        return false;
+      }
+      __nanosleep(32);
+    }
+  }
+  __threadfence();
+  return true;
+}
+
+// ---- 1. block-state reduction: ReLU(K)^T [V | 1] accumulated over the tiles of each segment ----
 namespace st {
 constexpr int kStages = 3;
 constexpr int kKBytes = 2 * kAtomBytes;          // K tile: 128 tokens x 128 features (two atoms)
 constexpr int kStageBytes = 2 * kKBytes;         // K + V
-constexpr int kOnesOff = kStages * kStageBytes;  // 16 KB of bf16 ones: B operand of the z column
-constexpr int kBarOff = kOnesOff + kAtomBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;
+constexpr int kOnesOff = kStages * kStageBytes;  // 16 token rows of bf16 ones: B operand of the z column
+constexpr int kOnesBytes = 2048;
+constexpr int kRegionBytes = kOnesOff + kOnesBytes;
+constexpr int kNumBars = 14;
+
+struct Bars {
+  uint64_t* full;   // [3] TMA landed (K and V)
+  uint64_t* relu;   // [3] ReLU(K) written back
+  uint64_t* empty;  // [3] MMAs reading the stage retired
+  uint64_t* accf;   // [2] accumulator holds a finished segment piece
+  uint64_t* acce;   // [2] accumulator drained by the epilogue
+  uint64_t* done;   // every MMA retired
+};
+__device__ __forceinline__ Bars bars_at(uint64_t* p) { return Bars{p, p + 3, p + 6, p + 9, p + 11, p + 13}; }
+__device__ __forceinline__ void init_bars(const Bars& b) {
+  for (int i = 0; i < kStages; ++i) {
+    mbar_init(&b.full[i], 1);
+    mbar_init(&b.relu[i], 4);
+    mbar_init(&b.empty[i], 1);
+  }
+  for (int a = 0; a < 2; ++a) {
+    mbar_init(&b.accf[a], 1);
+    mbar_init(&b.acce[a], 4);
+  }
+  mbar_init(b.done, 1);
+}
+// shared memory the MMA reads as constants: ones for the z column; zeros for features >= 64 when D <= 64
+__device__ __forceinline__ void init_smem(uint8_t* smem, bool two_atoms, int nthreads) {
+  uint4* ones = reinterpret_cast<uint4*>(smem + kOnesOff);
+  const uint4 one = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  for (int i = threadIdx.x; i < kOnesBytes / 16; i += nthreads) ones[i] = one;
+  if (!two_atoms) {
+    for (int s = 0; s < kStages; ++s) {
+      uint4* kz = reinterpret_cast<uint4*>(smem + s * kStageBytes + kAtomBytes);
+      uint4* vz = reinterpret_cast<uint4*>(smem + s * kStageBytes + kKBytes + kAtomBytes);
+      for (int i = threadIdx.x; i < kAtomBytes / 16; i += nthreads) {
+        kz[i] = make_uint4(0, 0, 0, 0);
+        vz[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+}
+
+// Producer. `wait_first`: K and V (and the partial slots) may belong to the previous kernel in the
+// stream, so nothing is touched before griddepcontrol.wait. Returns once every stage it filled has
+// been consumed by the MMAs, so the caller may reuse the stage memory.
+__device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb, long long te,
+                        bool two_atoms, bool wait_first, uint32_t* status) {
+  const uint64_t pol = policy_evict_first();
+  const uint32_t tx = two_atoms ? 2u * kKBytes : static_cast<uint32_t>(kKBytes);
+  if (wait_first) griddep_wait();
+  int k = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const TileCoord c = tile_coord(t, geo);
+    const int s = k % kStages;
+    if (!mbar_wait(&b.empty[s], ((k / kStages) & 1) ^ 1, status, 0x0100u | s)) break;
+    const bool lst = use_last_map(c, geo);
+    const CUtensorMap* mk = lst ? m.a_last : m.a_main;
+    const CUtensorMap* mv = lst ? m.b_last : m.b_main;
+    const int cb = lst ? 0 : c.blk;
+    uint8_t* stg = smem + s * kStageBytes;
+    mbar_expect_tx(&b.full[s], tx);
+    tma_load_4d(stg, mk, &b.full[s], 0, c.tok0, cb, c.bh, pol);
+    tma_load_4d(stg + kKBytes, mv, &b.full[s], 0, c.tok0, cb, c.bh, pol);
+    if (two_atoms) {
+      tma_load_4d(stg + kAtomBytes, mk, &b.full[s], 64, c.tok0, cb, c.bh, pol);
+      tma_load_4d(stg + kKBytes + kAtomBytes, mv, &b.full[s], 64, c.tok0, cb, c.bh, pol);
+    }
+  }
+  for (int j = (k > kStages ? k - kStages : 0); j < k; ++j)
+    mbar_wait(&b.empty[j % kStages], (j / kStages) & 1, status, 0x0180u);
+}
+
+__device__ void relu_role(uint8_t* smem, const Bars& b, long long tb, long long te, bool two_atoms, int r, int lane,
+                          uint32_t* status) {
+  const int nchunks = (two_atoms ? kKBytes : kAtomBytes) / 16;
+  int k = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const int s = k % kStages;
+    bool ok = mbar_wait(&b.full[s], (k / kStages) & 1, status, 0x0200u | s);
+    if (!warp_all(ok)) break;
+    relu_tile_inplace(smem + s * kStageBytes, nchunks, r);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b.relu[s]);
+  }
+}
+
+__device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, uint32_t tmem,
+                         uint32_t* status) {
+  constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, true, true);
+  constexpr uint32_t kIdescZ = idesc_bf16_f32(128, 16, true, true);
+  const uint64_t od = sdesc_sw128(smem_u32(smem + kOnesOff), kAtomBytes, 1024);  // same 16 rows of ones each step
+  int k = 0, j = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const TileCoord c = tile_coord(t, geo);
+    const bool first = (t == tb) || c.tok0 == 0;
+    const bool end = c.last || t == te - 1;
+    const int a = j & 1;
+    const int s = k % kStages;
+    const uint32_t ph = (k / kStages) & 1;
+    if (first && !mbar_wait(&b.acce[a], ((j >> 1) & 1) ^ 1, status, 0x0300u | a)) break;
+    if (!mbar_wait(&b.full[s], ph, status, 0x0310u | s)) break;
+    if (!mbar_wait(&b.relu[s], ph, status, 0x0320u | s)) break;
+    tc_fence_after();
+    const uint32_t kb = smem_u32(smem + s * kStageBytes);
+    const uint32_t vb = kb + kKBytes;
+    const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk) {
+      // 16 tokens per MMA: two groups of 8 token rows (128 B each) -> +2048 B per step
+      const uint64_t ad = sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024);
+      const uint64_t bd = sdesc_sw128(vb + kk * 2048, kAtomBytes, 1024);
+      const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+      mma_bf16(dacc, ad, bd, kIdescS, acc);         // S^T columns: ReLU(K)^T V
+      mma_bf16(dacc + 128, ad, od, kIdescZ, acc);   // z column: ReLU(K)^T 1
+    }
+    mma_commit(&b.empty[s]);
+    if (end) {
+      mma_commit(&b.accf[a]);
+      ++j;
+    }
+  }
+  mma_commit(b.done);
+  mbar_wait(b.done, 0, status, 0x03F0u);
+}
+
+// Epilogue: warp w drains TMEM lanes 32w..32w+31 (key feature d) into the partial slot g + segment,
+// and records which CTAs hold a segment's first and last tile.
+// With `slot_ready`, every flushed slot is then published for other CTAs (value `tag`): the four
+// warps meet on the CTA barrier `flushed` (count 4) and warp 0 releases the slot's flag.
+__device__ void epilogue_role(const Bars& b, const Geom& geo, long long tb, long long te, uint32_t tmem, int g,
+                              int warp, int lane, float* __restrict__ partials, int2* __restrict__ segcta,
+                              uint64_t* slot_ready, uint64_t* flushed, uint64_t tag, uint32_t* status) {
+  const int d = warp * 32 + lane;
+  int j = 0;
+  for (long long t = tb; t < te; ++t) {
+    const TileCoord c = tile_coord(t, geo);
+    if (!(c.last || t == te - 1)) continue;
+    const int a = j & 1;
+    bool ok = mbar_wait(&b.accf[a], (j >> 1) & 1, status, 0x0400u | a);
+    if (!warp_all(ok)) break;
+    tc_fence_after();
+    const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(a * 256);
+    float* dst = partials + static_cast<size_t>(g + c.seg) * (kPartRows * kDPad);
+    // two halves of 64 columns, each read with one wait (the register budget holds 64 values)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t rr[2][32];
+      uint32_t zr = 0;
+      tmem_ld_x32(ta + h * 64, rr[0]);
+      tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+      if (h == 1) tmem_ld_x1(ta + 128, zr);
+      tmem_wait_ld();
+      if (h == 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.acce[a]);  // the accumulator is free once the values are in registers
+      }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) dst[(h * 64 + cc * 32 + jj) * kDPad + d] = __uint_as_float(rr[cc][jj]);
+      if (h == 1) dst[kZRow * kDPad + d] = __uint_as_float(zr);
+    }
+    if (warp == 0 && lane == 0) {
+      if (t - c.tok0 / kTile >= tb) segcta[c.seg].x = g;
+      if (c.last) segcta[c.seg].y = g;
+    }
+    if (slot_ready != nullptr) {
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        mbar_arrive(flushed);
+        // every warp sees this flush complete before it can arrive for the next one
+        const bool all_written = mbar_wait(flushed, j & 1, status, 0x0480u);
+        if (warp == 0 && all_written) st_release_u64(slot_ready + g + c.seg, tag);
+      }
+    }
+    ++j;
+  }
+}
 }  // namespace st
 
-__global__ void __launch_bounds__(kThreads, 1)
-    state_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
-                      const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
-                      const Geom geo, float* __restrict__ partials, int2* __restrict__ segcta,
-                      uint32_t* status) {
-  using namespace st;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
-  uint64_t* full = bars;        // TMA landed (K and V)
-  uint64_t* relu = bars + 3;    // ReLU(K) written back
-  uint64_t* empty = bars + 6;   // MMAs reading the stage retired
-  uint64_t* accf = bars + 9;    // accumulator holds a finished segment
-  uint64_t* acce = bars + 11;   // accumulator drained by the epilogue
-  uint64_t* done = bars + 13;   // every MMA retired (teardown)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+// ---- 3. output GEMM ReLU(Q) [P | z]^T with the normalising divide in the epilogue ----
+namespace ot {
+constexpr int kStages = 3;
+constexpr int kQBytes = 2 * kAtomBytes;             // Q tile: 128 tokens x 128 features
+constexpr int kBOff = kStages * kQBytes;            // two prefix tiles (double-buffered)
+constexpr int kBAtomBytes = kPTileRows * 128;       // 144 rows x 128 B
+constexpr int kOOff = kBOff + 2 * kPTileBytes;      // output staging, one 8 KB slice per warp
+constexpr int kOWarpBytes = 2 * 32 * 128;
+constexpr int kRegionBytes = kOOff + 4 * kOWarpBytes;
+constexpr int kNumBars = 18;
+static_assert(kBOff % 1024 == 0 && kOOff % 1024 == 0 && kBAtomBytes % 1024 == 0, "1024-B atoms");
 
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int g = blockIdx.x;
-  const long long tb = tile_begin(g, geo);
-  const long long te = tile_begin(g + 1, geo);
-  const bool two_atoms = geo.D > 64;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&relu[i], 4);
-      mbar_init(&empty[i], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&accf[a], 1);
-      mbar_init(&acce[a], 4);
-    }
-    mbar_init(done, 1);
-    fence_mbar_init();
+struct Bars {
+  uint64_t* qfull;   // [3]
+  uint64_t* qrelu;   // [3]
+  uint64_t* qempty;  // [3]
+  uint64_t* bfull;   // [2]
+  uint64_t* bempty;  // [2]
+  uint64_t* accf;    // [2]
+  uint64_t* acce;    // [2]
+  uint64_t* done;
+};
+__device__ __forceinline__ Bars bars_at(uint64_t* p) {
+  return Bars{p, p + 3, p + 6, p + 9, p + 11, p + 13, p + 15, p + 17};
+}
+__device__ __forceinline__ void init_bars(const Bars& b) {
+  for (int i = 0; i < kStages; ++i) {
+    mbar_init(&b.qfull[i], 1);
+    mbar_init(&b.qrelu[i], 4);
+    mbar_init(&b.qempty[i], 1);
   }
-  {
-    uint4* ones = reinterpret_cast<uint4*>(smem + kOnesOff);
-    const uint4 one = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-    for (int i = threadIdx.x; i < kAtomBytes / 16; i += kThreads) ones[i] = one;
-    if (!two_atoms) {  // features 64..127 never loaded: keep them zero
-      for (int s = 0; s < kStages; ++s) {
-        uint4* kz = reinterpret_cast<uint4*>(smem + s * kStageBytes + kAtomBytes);
-        uint4* vz = reinterpret_cast<uint4*>(smem + s * kStageBytes + kKBytes + kAtomBytes);
-        for (int i = threadIdx.x; i < kAtomBytes / 16; i += kThreads) {
-          kz[i] = make_uint4(0, 0, 0, 0);
-          vz[i] = make_uint4(0, 0, 0, 0);
+  for (int a = 0; a < 2; ++a) {
+    mbar_init(&b.bfull[a], 1);
+    mbar_init(&b.bempty[a], 1);
+    mbar_init(&b.accf[a], 1);
+    mbar_init(&b.acce[a], 4);
+  }
+  mbar_init(b.done, 1);
+}
+
+__device__ __forceinline__ void load_q(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long t,
+                                       int s, bool two_atoms, uint64_t pol) {
+  const TileCoord c = tile_coord(t, geo);
+  const bool lst = use_last_map(c, geo);
+  const CUtensorMap* mq = lst ? m.a_last : m.a_main;
+  const int cb = lst ? 0 : c.blk;
+  uint8_t* stg = smem + s * kQBytes;
+  mbar_expect_tx(&b.qfull[s], two_atoms ? static_cast<uint32_t>(kQBytes) : static_cast<uint32_t>(kAtomBytes));
+  tma_load_4d(stg, mq, &b.qfull[s], 0, c.tok0, cb, c.bh, pol);
+  if (two_atoms) tma_load_4d(stg + kAtomBytes, mq, &b.qfull[s], 64, c.tok0, cb, c.bh, pol);
+}
+
+// Q was final before the state reduction ran, so the first stages can fill before the prefix
+// exists. Returns how many tiles were issued.
+__device__ int prefill(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb, long long te,
+                       bool two_atoms) {
+  const uint64_t pol = policy_evict_first();
+  const int pre = static_cast<int>(te - tb < kStages ? te - tb : kStages);
+  for (int i = 0; i < pre; ++i) load_q(smem, b, m, geo, tb + i, i, two_atoms, pol);
+  return pre;
+}
+
+// The rest of the producer: prefix tiles (read only once the prefix is complete) and the Q tiles
+// after the prefilled ones.
+// With `combined` (single-launch kernel, one block per head), a head's prefix tile is loaded only
+// once every CTA covering the head has published its share of the combine (value `tag`).
+__device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb, long long te,
+                        int pre, bool two_atoms, const uint8_t* __restrict__ ptiles, const uint64_t* combined,
+                        uint64_t tag, uint32_t* status) {
+  const uint64_t pol = policy_evict_first();
+  int k = 0, j = 0, prev = -1;
+  bool ok = true;
+  for (long long t = tb; t < te && ok; ++t, ++k) {
+    const TileCoord c = tile_coord(t, geo);
+    if (c.seg != prev) {
+      const int bb = j & 1;
+      if (combined != nullptr) {
+        const long long f = seg_first_tile(c.seg, geo);
+        const int g0 = cta_of_tile(f, geo), g1 = cta_of_tile(f + seg_ntiles(c.seg, geo) - 1, geo);
+        if (!wait_flags(combined, g0 + c.seg, g1 + c.seg, tag, status, 0x2200u)) break;
+        fence_proxy_async_global();  // prefix tile written by other CTAs -> bulk copy below
+      }
+      if (!mbar_wait(&b.bempty[bb], ((j >> 1) & 1) ^ 1, status, 0x1100u | bb)) break;
+      mbar_expect_tx(&b.bfull[bb], kPTileBytes);
+      bulk_load(smem + kBOff + bb * kPTileBytes, ptiles + static_cast<size_t>(c.seg) * kPTileBytes, kPTileBytes,
+                &b.bfull[bb]);
+      ++j;
+      prev = c.seg;
+    }
+    if (k >= pre) {
+      const int s = k % kStages;
+      if (!mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) break;
+      load_q(smem, b, m, geo, t, s, two_atoms, pol);
+    }
+  }
+  for (int i = (k > kStages ? k - kStages : 0); i < (k > pre ? k : pre); ++i)
+    mbar_wait(&b.qfull[i % kStages], (i / kStages) & 1, status, 0x1180u);
+  for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&b.bfull[i & 1], (i >> 1) & 1, status, 0x1190u);
+}
+
+__device__ void relu_role(uint8_t* smem, const Bars& b, long long tb, long long te, bool two_atoms, int r, int lane,
+                          uint32_t* status) {
+  const int nchunks = (two_atoms ? kQBytes : kAtomBytes) / 16;
+  int k = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const int s = k % kStages;
+    bool ok = mbar_wait(&b.qfull[s], (k / kStages) & 1, status, 0x1200u | s);
+    if (!warp_all(ok)) break;
+    relu_tile_inplace(smem + s * kQBytes, nchunks, r);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b.qrelu[s]);
+  }
+}
+
+__device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, bool two_atoms,
+                         uint32_t tmem, uint32_t* status) {
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, kPTileRows, false, false);
+  const int ksteps = two_atoms ? 8 : 4;
+  int k = 0, j = 0, prev = -1, bb = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const TileCoord c = tile_coord(t, geo);
+    if (c.seg != prev) {
+      bb = j & 1;
+      if (!mbar_wait(&b.bfull[bb], (j >> 1) & 1, status, 0x1300u | bb)) break;
+      ++j;
+      prev = c.seg;
+    }
+    const int s = k % kStages;
+    const uint32_t ph = (k / kStages) & 1;
+    const int a = k & 1;
+    if (!mbar_wait(&b.qfull[s], ph, status, 0x1310u | s)) break;
+    if (!mbar_wait(&b.qrelu[s], ph, status, 0x1320u | s)) break;
+    if (!mbar_wait(&b.acce[a], ((k >> 1) & 1) ^ 1, status, 0x1330u | a)) break;
+    tc_fence_after();
+    const uint32_t qb = smem_u32(smem + s * kQBytes);
+    const uint32_t bbase = smem_u32(smem + kBOff + bb * kPTileBytes);
+    const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
+    for (int kk = 0; kk < ksteps; ++kk) {
+      // 16 features per MMA: +32 B inside the 128-B swizzle row, next atom after 4 steps
+      const uint64_t ad = sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = sdesc_sw128(bbase + (kk >> 2) * kBAtomBytes + (kk & 3) * 32, 16, 1024);
+      mma_bf16(dacc, ad, bd, kIdescO, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&b.qempty[s]);
+    mma_commit(&b.accf[a]);
+    if (c.last || t == te - 1) mma_commit(&b.bempty[bb]);
+  }
+  mma_commit(b.done);
+  mbar_wait(b.done, 0, status, 0x13F0u);
+}
+
+// Epilogue: warp w owns tokens 32w..32w+31 of the tile (TMEM lanes); numerator columns times
+// 1 / (denominator + eps), bf16, swizzled staging, TMA store clipped to the block.
+__device__ void epilogue_role(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
+                              long long te, bool two_atoms, uint32_t tmem, int warp, int lane, float eps,
+                              uint32_t* status) {
+  uint8_t* ob = smem + kOOff + warp * kOWarpBytes;
+  const int ncc = two_atoms ? 4 : 2;
+  int k = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const TileCoord c = tile_coord(t, geo);
+    const int a = k & 1;
+    bool ok = mbar_wait(&b.accf[a], (k >> 1) & 1, status, 0x1400u | a);
+    if (!warp_all(ok)) break;
+    tc_fence_after();
+    const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(a * 256);
+    // two halves of 64 columns, each read with one wait (the register budget holds 64 values)
+    uint32_t dr;
+    tmem_ld_x1(ta + kZRow, dr);
+    float inv = 0.f;
+    for (int h = 0; h < 2; ++h) {
+      if (2 * h >= ncc) break;
+      uint32_t rr[2][32];
+      tmem_ld_x32(ta + h * 64, rr[0]);
+      tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+      tmem_wait_ld();
+      if (h == 0) {
+        inv = __frcp_rn(__uint_as_float(dr) + eps);
+        if (lane == 0) bulk_wait_read_all();  // the previous store has finished reading the slice
+        __syncwarp();
+      }
+      if (2 * h + 2 >= ncc) {  // last half read: the accumulator is free
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.acce[a]);
+      }
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 0]) * inv, __uint_as_float(rr[cc][8 * mm + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 2]) * inv, __uint_as_float(rr[cc][8 * mm + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 4]) * inv, __uint_as_float(rr[cc][8 * mm + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 6]) * inv, __uint_as_float(rr[cc][8 * mm + 7]) * inv);
+          const int chunk = (2 * h + cc) * 4 + mm;  // 16-byte chunk of the 256-byte output row
+          uint8_t* dst = ob + (chunk >> 3) * 4096 + lane * 128 + (((chunk & 7) ^ (lane & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = w;
         }
       }
     }
     fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int blen = (c.blk == geo.nblk - 1) ? geo.Llast : geo.L;
+      const int row0 = c.tok0 + warp * 32;
+      if (row0 < blen) {
+        const bool lst = use_last_map(c, geo);
+        const CUtensorMap* mo = lst ? m.b_last : m.b_main;
+        const int cb = lst ? 0 : c.blk;
+        tma_store_4d(mo, ob, 0, row0, cb, c.bh);
+        if (two_atoms) tma_store_4d(mo, ob + 4096, 64, row0, cb, c.bh);
+        bulk_commit();
+      }
+    }
   }
+  if (lane == 0) bulk_wait_all();
+}
+}  // namespace ot
+
+// ---- common prologue / epilogue of the persistent kernels ----
+__device__ __forceinline__ void prefetch_maps(const Maps4& m) {
+  prefetch_tmap(m.a_main);
+  prefetch_tmap(m.a_last);
+  prefetch_tmap(m.b_main);
+  prefetch_tmap(m.b_last);
+}
+__device__ __forceinline__ uint32_t persistent_setup(uint32_t* tmem_slot, int warp) {
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kWarpProducer && lane == 0) {
-    prefetch_tmap(&k_main);
-    prefetch_tmap(&v_main);
-    prefetch_tmap(&k_last);
-    prefetch_tmap(&v_last);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) griddep_launch_dependents();
-
-  if (warp == kWarpProducer) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      const uint32_t tx = two_atoms ? 2u * kKBytes : static_cast<uint32_t>(kKBytes);
-      // K, V may come from the previous kernel in the stream, and the partial slots written below
-      // may still be read by the previous call's scan: nothing is touched before this wait.
-      griddep_wait();
-      int k = 0;
-      for (long long t = tb; t < te; ++t, ++k) {
-        const TileCoord c = tile_coord(t, geo);
-        const int s = k % kStages;
-        if (!mbar_wait(&empty[s], ((k / kStages) & 1) ^ 1, status, 0x0100u | s)) break;
-        const bool lst = use_last_map(c, geo);
-        const CUtensorMap* mk = lst ? &k_last : &k_main;
-        const CUtensorMap* mv = lst ? &v_last : &v_main;
-        const int cb = lst ? 0 : c.blk;
-        uint8_t* stg = smem + s * kStageBytes;
-        mbar_expect_tx(&full[s], tx);
-        tma_load_4d(stg, mk, &full[s], 0, c.tok0, cb, c.bh, pol);
-        tma_load_4d(stg + kKBytes, mv, &full[s], 0, c.tok0, cb, c.bh, pol);
-        if (two_atoms) {
-          tma_load_4d(stg + kAtomBytes, mk, &full[s], 64, c.tok0, cb, c.bh, pol);
-          tma_load_4d(stg + kKBytes + kAtomBytes, mv, &full[s], 64, c.tok0, cb, c.bh, pol);
-        }
-      }
-      // the loads issued last into each stage land before the CTA can exit
-      for (int j = (k > kStages ? k - kStages : 0); j < k; ++j)
-        mbar_wait(&full[j % kStages], (j / kStages) & 1, status, 0x0180u);
-    }
-  } else if (warp >= 4 && warp < 8) {
-    const int r = threadIdx.x - 128;
-    const int nchunks = (two_atoms ? kKBytes : kAtomBytes) / 16;
-    int k = 0;
-    for (long long t = tb; t < te; ++t, ++k) {
-      const int s = k % kStages;
-      bool ok = mbar_wait(&full[s], (k / kStages) & 1, status, 0x0200u | s);
-      if (!warp_all(ok)) break;
-      relu_tile_inplace(smem + s * kStageBytes, nchunks, r);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&relu[s]);
-    }
-  } else if (warp == kWarpMma) {
-    if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, true, true);
-      constexpr uint32_t kIdescZ = idesc_bf16_f32(128, 16, true, true);
-      const uint32_t ones = smem_u32(smem + kOnesOff);
-      int k = 0, j = 0;
-      for (long long t = tb; t < te; ++t, ++k) {
-        const TileCoord c = tile_coord(t, geo);
-        const bool first = (t == tb) || c.tok0 == 0;
-        const bool end = c.last || t == te - 1;
-        const int a = j & 1;
-        const int s = k % kStages;
-        const uint32_t ph = (k / kStages) & 1;
-        if (first && !mbar_wait(&acce[a], ((j >> 1) & 1) ^ 1, status, 0x0300u | a)) break;
-        if (!mbar_wait(&full[s], ph, status, 0x0310u | s)) break;
-        if (!mbar_wait(&relu[s], ph, status, 0x0320u | s)) break;
-        tc_fence_after();
-        const uint32_t kb = smem_u32(smem + s * kStageBytes);
-        const uint32_t vb = kb + kKBytes;
-        const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          // 16 tokens per MMA: two groups of 8 token rows (128 B each) -> +2048 B per step
-          const uint64_t ad = sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024);
-          const uint64_t bd = sdesc_sw128(vb + kk * 2048, kAtomBytes, 1024);
-          const uint64_t od = sdesc_sw128(ones + kk * 2048, kAtomBytes, 1024);
-          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          mma_bf16(dacc, ad, bd, kIdescS, acc);         // S^T columns: ReLU(K)^T V
-          mma_bf16(dacc + 128, ad, od, kIdescZ, acc);   // z column: ReLU(K)^T 1
-        }
-        mma_commit(&empty[s]);
-        if (end) {
-          mma_commit(&accf[a]);
-          ++j;
-        }
-      }
-      mma_commit(done);
-      mbar_wait(done, 0, status, 0x03F0u);
-    }
-  } else {
-    // epilogue: warp w drains TMEM lanes 32w..32w+31 (key feature d) into the partial slot
-    const int d = warp * 32 + lane;
-    int j = 0;
-    for (long long t = tb; t < te; ++t) {
-      const TileCoord c = tile_coord(t, geo);
-      if (!(c.last || t == te - 1)) continue;
-      const int a = j & 1;
-      bool ok = mbar_wait(&accf[a], (j >> 1) & 1, status, 0x0400u | a);
-      if (!warp_all(ok)) break;
-      tc_fence_after();
-      const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(a * 256);
-      float* dst = partials + static_cast<size_t>(g + c.seg) * (kPartRows * kDPad);
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld_x32(ta + cc * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) dst[(cc * 32 + jj) * kDPad + d] = __uint_as_float(r[jj]);
-      }
-      uint32_t zr;
-      tmem_ld_x1(ta + 128, zr);
-      tmem_wait_ld();
-      dst[kZRow * kDPad + d] = __uint_as_float(zr);
-      if (warp == 0 && lane == 0) {  // which CTAs hold the first and the last tile of the segment
-        if (t - c.tok0 / kTile >= tb) segcta[c.seg].x = g;
-        if (c.last) segcta[c.seg].y = g;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[a]);
-      ++j;
-    }
-  }
-
+  return *tmem_slot;
+}
+__device__ __forceinline__ void persistent_teardown(uint32_t tmem, int warp) {
+  tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
     tc_fence_after();
@@ -263,226 +556,85 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// 3. output GEMM with the normalising divide in the epilogue (bf16 in/out)
+// stand-alone kernels
 // ------------------------------------------------------------------------------------------
-namespace ot {
-constexpr int kStages = 3;
-constexpr int kQBytes = 2 * kAtomBytes;             // Q tile: 128 tokens x 128 features
-constexpr int kBOff = kStages * kQBytes;            // two prefix tiles (double-buffered)
-constexpr int kBAtomBytes = kPTileRows * 128;       // 144 rows x 128 B
-constexpr int kOOff = kBOff + 2 * kPTileBytes;      // output staging, one 8 KB slice per warp
-constexpr int kOWarpBytes = 2 * 32 * 128;
-constexpr int kBarOff = kOOff + 4 * kOWarpBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;
-static_assert(kBOff % 1024 == 0 && kOOff % 1024 == 0 && kBAtomBytes % 1024 == 0, "1024-B atoms");
-}  // namespace ot
+constexpr int kStateSmem = st::kRegionBytes + 1024 + 256 + 1024;   // region, barriers, alignment slack
+constexpr int kOutSmem = ot::kRegionBytes + 1024 + 256 + 1024;
 
 __global__ void __launch_bounds__(kThreads, 1)
-    out_bf16_kernel(const __grid_constant__ CUtensorMap q_main, const __grid_constant__ CUtensorMap q_last,
-                    const __grid_constant__ CUtensorMap o_main, const __grid_constant__ CUtensorMap o_last,
-                    const Geom geo, const uint8_t* __restrict__ ptiles, const float eps, uint32_t* status) {
-  using namespace ot;
+    state_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
+                      const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
+                      const Geom geo, float* __restrict__ partials, int2* __restrict__ segcta,
+                      uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
-  uint64_t* qfull = bars;
-  uint64_t* qrelu = bars + 3;
-  uint64_t* qempty = bars + 6;
-  uint64_t* bfull = bars + 9;
-  uint64_t* bempty = bars + 11;
-  uint64_t* accf = bars + 13;
-  uint64_t* acce = bars + 15;
-  uint64_t* done = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
-
+  uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + st::kRegionBytes);
+  const st::Bars b = st::bars_at(barmem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + st::kNumBars);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
   const long long tb = tile_begin(g, geo);
   const long long te = tile_begin(g + 1, geo);
   const bool two_atoms = geo.D > 64;
-
+  const Maps4 m{&k_main, &k_last, &v_main, &v_last};
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&qfull[i], 1);
-      mbar_init(&qrelu[i], 4);
-      mbar_init(&qempty[i], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&bfull[a], 1);
-      mbar_init(&bempty[a], 1);
-      mbar_init(&accf[a], 1);
-      mbar_init(&acce[a], 4);
-    }
-    mbar_init(done, 1);
+    st::init_bars(b);
     fence_mbar_init();
   }
-  if (warp == kWarpMma) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
-  if (warp == kWarpProducer && lane == 0) {
-    prefetch_tmap(&q_main);
-    prefetch_tmap(&q_last);
-    prefetch_tmap(&o_main);
-    prefetch_tmap(&o_last);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
+  st::init_smem(smem, two_atoms, kThreads);
+  if (warp == kWarpProducer && lane == 0) prefetch_maps(m);
+  const uint32_t tmem = persistent_setup(tmem_slot, warp);
   if (threadIdx.x == 0) griddep_launch_dependents();
+  if (warp == kWarpProducer) {
+    if (lane == 0) st::produce(smem, b, m, geo, tb, te, two_atoms, true, status);
+  } else if (warp >= 4 && warp < 8) {
+    st::relu_role(smem, b, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) st::mma_role(smem, b, geo, tb, te, tmem, status);
+  } else {
+    st::epilogue_role(b, geo, tb, te, tmem, g, warp, lane, partials, segcta, nullptr, nullptr, 0, status);
+  }
+  persistent_teardown(tmem, warp);
+}
 
+__global__ void __launch_bounds__(kThreads, 1)
+    out_bf16_kernel(const __grid_constant__ CUtensorMap q_main, const __grid_constant__ CUtensorMap q_last,
+                    const __grid_constant__ CUtensorMap o_main, const __grid_constant__ CUtensorMap o_last,
+                    const Geom geo, const uint8_t* __restrict__ ptiles, const float eps, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + ot::kRegionBytes);
+  const ot::Bars b = ot::bars_at(barmem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + ot::kNumBars);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.x;
+  const long long tb = tile_begin(g, geo);
+  const long long te = tile_begin(g + 1, geo);
+  const bool two_atoms = geo.D > 64;
+  const Maps4 m{&q_main, &q_last, &o_main, &o_last};
+  if (threadIdx.x == 0) {
+    ot::init_bars(b);
+    fence_mbar_init();
+  }
+  if (warp == kWarpProducer && lane == 0) prefetch_maps(m);
+  const uint32_t tmem = persistent_setup(tmem_slot, warp);
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == kWarpProducer) {
     if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      const uint32_t tx = two_atoms ? static_cast<uint32_t>(kQBytes) : static_cast<uint32_t>(kAtomBytes);
-      auto load_q = [&](long long t, int s) {
-        const TileCoord c = tile_coord(t, geo);
-        const bool lst = use_last_map(c, geo);
-        const CUtensorMap* mq = lst ? &q_last : &q_main;
-        const int cb = lst ? 0 : c.blk;
-        uint8_t* stg = smem + s * kQBytes;
-        mbar_expect_tx(&qfull[s], tx);
-        tma_load_4d(stg, mq, &qfull[s], 0, c.tok0, cb, c.bh, pol);
-        if (two_atoms) tma_load_4d(stg + kAtomBytes, mq, &qfull[s], 64, c.tok0, cb, c.bh, pol);
-      };
-      // Q was final before the state kernel ran, so the first stages fill while the scan runs;
-      // the prefix tiles are read only after the scan grid has completed.
-      const int pre = static_cast<int>(te - tb < kStages ? te - tb : kStages);
-      for (int i = 0; i < pre; ++i) load_q(tb + i, i);
-      griddep_wait();
-      int k = 0, j = 0, prev = -1;
-      for (long long t = tb; t < te; ++t, ++k) {
-        const TileCoord c = tile_coord(t, geo);
-        if (c.seg != prev) {
-          const int bb = j & 1;
-          if (!mbar_wait(&bempty[bb], ((j >> 1) & 1) ^ 1, status, 0x1100u | bb)) break;
-          mbar_expect_tx(&bfull[bb], kPTileBytes);
-          bulk_load(smem + kBOff + bb * kPTileBytes, ptiles + static_cast<size_t>(c.seg) * kPTileBytes,
-                    kPTileBytes, &bfull[bb]);
-          ++j;
-          prev = c.seg;
-        }
-        if (k >= pre) {
-          const int s = k % kStages;
-          if (!mbar_wait(&qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) break;
-          load_q(t, s);
-        }
-      }
-      for (int i = (k > kStages ? k - kStages : 0); i < (k > pre ? k : pre); ++i)
-        mbar_wait(&qfull[i % kStages], (i / kStages) & 1, status, 0x1180u);
-      for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&bfull[i & 1], (i >> 1) & 1, status, 0x1190u);
+      const int pre = ot::prefill(smem, b, m, geo, tb, te, two_atoms);
+      griddep_wait();  // the prefix tiles come from the scan grid
+      ot::produce(smem, b, m, geo, tb, te, pre, two_atoms, ptiles, nullptr, 0, status);
     }
   } else if (warp >= 4 && warp < 8) {
-    const int r = threadIdx.x - 128;
-    const int nchunks = (two_atoms ? kQBytes : kAtomBytes) / 16;
-    int k = 0;
-    for (long long t = tb; t < te; ++t, ++k) {
-      const int s = k % kStages;
-      bool ok = mbar_wait(&qfull[s], (k / kStages) & 1, status, 0x1200u | s);
-      if (!warp_all(ok)) break;
-      relu_tile_inplace(smem + s * kQBytes, nchunks, r);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qrelu[s]);
-    }
+    ot::relu_role(smem, b, tb, te, two_atoms, threadIdx.x - 128, lane, status);
   } else if (warp == kWarpMma) {
-    if (lane == 0) {
-      constexpr uint32_t kIdescO = idesc_bf16_f32(128, kPTileRows, false, false);
-      const int ksteps = two_atoms ? 8 : 4;
-      int k = 0, j = 0, prev = -1, bb = 0;
-      for (long long t = tb; t < te; ++t, ++k) {
-        const TileCoord c = tile_coord(t, geo);
-        if (c.seg != prev) {
-          bb = j & 1;
-          if (!mbar_wait(&bfull[bb], (j >> 1) & 1, status, 0x1300u | bb)) break;
-          ++j;
-          prev = c.seg;
-        }
-        const int s = k % kStages;
-        const uint32_t ph = (k / kStages) & 1;
-        const int a = k & 1;
-        if (!mbar_wait(&qfull[s], ph, status, 0x1310u | s)) break;
-        if (!mbar_wait(&qrelu[s], ph, status, 0x1320u | s)) break;
-        if (!mbar_wait(&acce[a], ((k >> 1) & 1) ^ 1, status, 0x1330u | a)) break;
-        tc_fence_after();
-        const uint32_t qb = smem_u32(smem + s * kQBytes);
-        const uint32_t bbase = smem_u32(smem + kBOff + bb * kPTileBytes);
-        const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
-        for (int kk = 0; kk < ksteps; ++kk) {
-          // 16 features per MMA: +32 B inside the 128-B swizzle row, next atom after 4 steps
-          const uint64_t ad = sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(bbase + (kk >> 2) * kBAtomBytes + (kk & 3) * 32, 16, 1024);
-          mma_bf16(dacc, ad, bd, kIdescO, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&qempty[s]);
-        mma_commit(&accf[a]);
-        if (c.last || t == te - 1) mma_commit(&bempty[bb]);
-      }
-      mma_commit(done);
-      mbar_wait(done, 0, status, 0x13F0u);
-    }
+    if (lane == 0) ot::mma_role(smem, b, geo, tb, te, two_atoms, tmem, status);
   } else {
-    // epilogue: warp w owns tokens 32w..32w+31 of the tile (TMEM lanes)
-    uint8_t* ob = smem + kOOff + warp * kOWarpBytes;
-    const int ncc = two_atoms ? 4 : 2;
-    int k = 0;
-    for (long long t = tb; t < te; ++t, ++k) {
-      const TileCoord c = tile_coord(t, geo);
-      const int a = k & 1;
-      bool ok = mbar_wait(&accf[a], (k >> 1) & 1, status, 0x1400u | a);
-      if (!warp_all(ok)) break;
-      tc_fence_after();
-      const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(a * 256);
-      uint32_t dr;
-      tmem_ld_x1(ta + kZRow, dr);
-      tmem_wait_ld();
-      const float inv = __frcp_rn(__uint_as_float(dr) + eps);
-      if (lane == 0) bulk_wait_read_all();  // the previous store has finished reading the slice
-      __syncwarp();
-      for (int cc = 0; cc < ncc; ++cc) {
-        uint32_t r[32];
-        tmem_ld_x32(ta + cc * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(r[8 * m + 0]) * inv, __uint_as_float(r[8 * m + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(r[8 * m + 2]) * inv, __uint_as_float(r[8 * m + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(r[8 * m + 4]) * inv, __uint_as_float(r[8 * m + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(r[8 * m + 6]) * inv, __uint_as_float(r[8 * m + 7]) * inv);
-          const int chunk = cc * 4 + m;  // 16-byte chunk of the 256-byte output row
-          uint8_t* dst = ob + (chunk >> 3) * 4096 + lane * 128 + (((chunk & 7) ^ (lane & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = w;
-        }
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&acce[a]);
-        const int blen = (c.blk == geo.nblk - 1) ? geo.Llast : geo.L;
-        const int row0 = c.tok0 + warp * 32;
-        if (row0 < blen) {
-          const bool lst = use_last_map(c, geo);
-          const CUtensorMap* mo = lst ? &o_last : &o_main;
-          const int cb = lst ? 0 : c.blk;
-          tma_store_4d(mo, ob, 0, row0, cb, c.bh);
-          if (two_atoms) tma_store_4d(mo, ob + 4096, 64, row0, cb, c.bh);
-          bulk_commit();
-        }
-      }
-    }
-    if (lane == 0) bulk_wait_all();
+    ot::epilogue_role(smem, b, m, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
   }
-
-  __syncthreads();
-  if (warp == kWarpMma) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
+  persistent_teardown(tmem, warp);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -516,16 +668,21 @@ __global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ pa
                                                     const int2* __restrict__ segcta, const Geom geo,
                                                     const float* S_in, const float* z_in, float* S_out,
                                                     float* z_out, uint8_t* __restrict__ ptiles,
-                                                    float* __restrict__ p32) {
+                                                    float* __restrict__ p32, const int ng_warps) {
   griddep_wait();  // partials come from the state kernel; prefix tiles may still be read before it
   griddep_launch_dependents();
-  extern __shared__ float4 s_scan[];   // [ng][32] warp totals, then [32] incoming cache
-  float4* s_base = s_scan + (blockDim.x >> 5) * 32;
+  // block (bh, rows e = blockIdx.y * R .. + R - 1): warp w handles row r = w / ng, block group j = w % ng
+  extern __shared__ float4 s_scan[];   // [R][ng][32] warp totals, then [R][32] incoming cache
+  const int ng = ng_warps;
+  const int R = (blockDim.x >> 5) / ng;
+  const int wr = threadIdx.x >> 5;
+  const int r = wr / ng;
   const int bh = blockIdx.x;
-  const int e = blockIdx.y;
+  const int e = blockIdx.y * R + r;
   const int q = threadIdx.x & 31;
-  const int j = threadIdx.x >> 5;
-  const int ng = blockDim.x >> 5;
+  const int j = wr - r * ng;
+  float4* s_tot = s_scan + r * ng * 32;
+  float4* s_base = s_scan + R * ng * 32 + r * 32;
   const int nblk = geo.nblk;
   const int D = geo.D;
   const int d0 = q * 4;
@@ -565,11 +722,11 @@ __global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ pa
   }
   float4 run = make_float4(base[0], base[1], base[2], base[3]);
   if (ng > 1) {
-    s_scan[j * 32 + q] = tot;
+    s_tot[j * 32 + q] = tot;
     if (j == 0) s_base[q] = run;
     __syncthreads();
     run = s_base[q];
-    for (int jj = 0; jj < j; ++jj) run = f4add(run, s_scan[jj * 32 + q]);
+    for (int jj = 0; jj < j; ++jj) run = f4add(run, s_tot[jj * 32 + q]);
   }
 
   // pass 2: running prefix, one prefix tile row chunk per block
@@ -610,6 +767,207 @@ __global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ pa
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         if (d0 + u < D) z_out[static_cast<size_t>(bh) * D + d0 + u] = r[u];
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 4. one launch for one-block problems (bidirectional forward, streaming cache step)
+// ------------------------------------------------------------------------------------------
+// State reduction -> combine -> output in one cooperative launch (every CTA resident, one per SM).
+// Each CTA reduces and then outputs the same contiguous tile range; heads are synchronised one by
+// one instead of with grid-wide barriers: a CTA publishes each partial slot it flushes; the CTAs
+// covering a head split that head's combine once all its slots are published, and publish their
+// share; a head's output starts once its combine is complete. Flags carry the workspace's launch
+// sequence number (header bytes 8..15, advanced by the last CTA to exit), so nothing needs resetting.
+// The stage memory of the reduction is reused by the output, whose first Q tiles load before the
+// combine.
+namespace fu {
+constexpr int kRegion = (st::kRegionBytes > ot::kRegionBytes) ? st::kRegionBytes : ot::kRegionBytes;
+constexpr int kSmem = kRegion + 512 + 1024;
+// shared memory free during the combine (between the prefilled Q stages and the output staging):
+// the cache transpose of up to 128 rows x 129 floats
+constexpr int kScratchOff = ot::kBOff;
+static_assert(kScratchOff + 128 * 129 * 4 <= ot::kOOff, "combine scratch overlaps the output staging");
+}  // namespace fu
+
+// This CTA's share of head bh's combine: rows [r0, r1) of the prefix tile (row e < 128: value
+// feature e of S; row 128: z; rows 129..143: zero), each row = S_in/z_in + the head's partial slots
+// of CTAs g0..g1, written as the bf16 B operand of the output GEMM and, when asked, to the cache.
+// The cache is [d][e] (key feature major) while a prefix row is one value feature e, so S_in and
+// S_out go through a shared-memory transpose `sS` to keep the global accesses coalesced.
+__device__ void combine_rows(const Geom& geo, const float* __restrict__ partials, int g0, int g1, const float* S_in,
+                             const float* z_in, float* S_out, float* z_out, uint8_t* __restrict__ ptiles, int bh,
+                             int r0, int r1, float* sS) {
+  const int D = geo.D;
+  const int e_hi = (r1 < D ? r1 : D);          // S rows of the share: [r0, e_hi)
+  const int ns = e_hi > r0 ? e_hi - r0 : 0;
+  const int ld = D + 1;                         // padded row of sS
+  if (S_in != nullptr && ns > 0) {
+    for (int i = threadIdx.x; i < D * ns; i += kThreads) {
+      const int d = i / ns, j = i - d * ns;     // consecutive threads: consecutive e of one key row d
+      sS[j * ld + d] = S_in[(static_cast<size_t>(bh) * D + d) * D + r0 + j];
+    }
+  }
+  __syncthreads();
+  for (int it = r0 * 32 + static_cast<int>(threadIdx.x); it < r1 * 32; it += kThreads) {
+    const int e = it >> 5;
+    const int d0 = (it & 31) * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (e < kPartRows) {
+      for (int gg = g0; gg <= g1; ++gg) {
+        const float4 p = *reinterpret_cast<const float4*>(
+            partials + (static_cast<size_t>(gg + bh) * kPartRows + e) * kDPad + d0);
+        acc[0] += p.x;
+        acc[1] += p.y;
+        acc[2] += p.z;
+        acc[3] += p.w;
+      }
+      if (e < D) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (d0 + u < D) {
+            if (S_in != nullptr) acc[u] += sS[(e - r0) * ld + d0 + u];
+            if (S_out != nullptr) sS[(e - r0) * ld + d0 + u] = acc[u];
+          }
+        }
+      }
+      if (e == kZRow) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (d0 + u < D) {
+            if (z_in != nullptr) acc[u] += z_in[static_cast<size_t>(bh) * D + d0 + u];
+          }
+        }
+        if (z_out != nullptr) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (d0 + u < D) z_out[static_cast<size_t>(bh) * D + d0 + u] = acc[u];
+        }
+      }
+    }
+    uint2 w;
+    w.x = pack_bf16x2(acc[0], acc[1]);
+    w.y = pack_bf16x2(acc[2], acc[3]);
+    const size_t off = static_cast<size_t>(bh) * kPTileBytes + (d0 >> 6) * (kPTileRows * 128) + e * 128 +
+                       ((((d0 & 63) >> 3) ^ (e & 7)) << 4) + (d0 & 7) * 2;
+    *reinterpret_cast<uint2*>(ptiles + off) = w;
+  }
+  __syncthreads();
+  if (S_out != nullptr && ns > 0) {
+    for (int i = threadIdx.x; i < D * ns; i += kThreads) {
+      const int d = i / ns, j = i - d * ns;
+      S_out[(static_cast<size_t>(bh) * D + d) * D + r0 + j] = sS[j * ld + d];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
+                      const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
+                      const __grid_constant__ CUtensorMap q_main, const __grid_constant__ CUtensorMap q_last,
+                      const __grid_constant__ CUtensorMap o_main, const __grid_constant__ CUtensorMap o_last,
+                      const Geom geo, float* __restrict__ partials, int2* __restrict__ segcta,
+                      uint64_t* __restrict__ slot_ready, uint64_t* __restrict__ combined,
+                      uint8_t* __restrict__ ptiles, const float* S_in, const float* z_in, float* S_out,
+                      float* z_out, const float eps, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_ok;
+  __shared__ uint64_t s_tag;
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + fu::kRegion);
+  const st::Bars sb = st::bars_at(barmem);
+  const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
+  uint64_t* flushed = barmem + st::kNumBars + ot::kNumBars;  // epilogue warps finished a slot (count 4)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flushed + 1);
+  uint64_t* seqp = reinterpret_cast<uint64_t*>(status + 2);  // header bytes 8..15: launch sequence number
+  uint32_t* gexit = status + 4;                              // header bytes 16..19: CTAs that finished
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.x;
+  const int G = gridDim.x;
+  const long long tb = tile_begin(g, geo);
+  const long long te = tile_begin(g + 1, geo);
+  const bool two_atoms = geo.D > 64;
+  const Maps4 mkv{&k_main, &k_last, &v_main, &v_last};
+  const Maps4 mqo{&q_main, &q_last, &o_main, &o_last};
+  if (threadIdx.x == 0) {
+    st::init_bars(sb);
+    ot::init_bars(ob);
+    mbar_init(flushed, 4);
+    fence_mbar_init();
+    s_ok = 1;
+    s_tag = ld_acquire_u64(seqp) + 1;
+  }
+  st::init_smem(smem, two_atoms, kThreads);
+  if (warp == kWarpProducer && lane == 0) {
+    prefetch_maps(mkv);
+    prefetch_maps(mqo);
+  }
+  const uint32_t tmem = persistent_setup(tmem_slot, warp);
+  const uint64_t tag = s_tag;
+
+  // phase 1: block states of this CTA's tiles; the producer then fills the first Q stages
+  int pre = 0;
+  if (warp == kWarpProducer) {
+    if (lane == 0) {
+      st::produce(smem, sb, mkv, geo, tb, te, two_atoms, false, status);
+      pre = ot::prefill(smem, ob, mqo, geo, tb, te, two_atoms);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    st::relu_role(smem, sb, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) st::mma_role(smem, sb, geo, tb, te, tmem, status);
+  } else {
+    st::epilogue_role(sb, geo, tb, te, tmem, g, warp, lane, partials, segcta, slot_ready, flushed, tag, status);
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // phase 2: this CTA's share of the combine of each head it covers, once all the head's slots exist
+  const int h0 = tile_coord(tb, geo).seg;
+  const int h1 = tile_coord(te - 1, geo).seg;
+  for (int h = h0; h <= h1; ++h) {
+    const long long f = seg_first_tile(h, geo);
+    const int g0 = cta_of_tile(f, geo), g1 = cta_of_tile(f + seg_ntiles(h, geo) - 1, geo);
+    if (threadIdx.x == 0 && s_ok && !wait_flags(slot_ready, g0 + h, g1 + h, tag, status, 0x2000u)) s_ok = 0;
+    __syncthreads();
+    if (s_ok) {  // whole rows per CTA, so each cache element belongs to exactly one CTA
+      const int n = g1 - g0 + 1, idx = g - g0;
+      combine_rows(geo, partials, g0, g1, S_in, z_in, S_out, z_out, ptiles, h, idx * kPTileRows / n,
+                   (idx + 1) * kPTileRows / n, reinterpret_cast<float*>(smem + fu::kScratchOff));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && s_ok) {
+      __threadfence();
+      st_release_u64(combined + g + h, tag);
+    }
+  }
+  fence_proxy_async_smem();  // the combine scratch is next written by TMA copies (async proxy)
+  __syncthreads();
+  tc_fence_after();
+
+  // phase 3: output of the same tiles, each head as soon as its combine is complete
+  if (s_ok) {
+    if (warp == kWarpProducer) {
+      if (lane == 0) ot::produce(smem, ob, mqo, geo, tb, te, pre, two_atoms, ptiles, combined, tag, status);
+    } else if (warp >= 4 && warp < 8) {
+      ot::relu_role(smem, ob, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+    } else if (warp == kWarpMma) {
+      if (lane == 0) ot::mma_role(smem, ob, geo, tb, te, two_atoms, tmem, status);
+    } else {
+      ot::epilogue_role(smem, ob, mqo, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
+    }
+  } else if (warp == kWarpProducer && lane == 0) {
+    for (int i = 0; i < pre; ++i) mbar_wait(&ob.qfull[i], 0, status, 0x2180u);  // prefilled loads land
+  }
+  persistent_teardown(tmem, warp);
+  // the last CTA out advances the launch sequence number for the next launch on this workspace
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(gexit, 1u) == static_cast<uint32_t>(G - 1)) {
+      *gexit = 0u;
+      st_release_u64(seqp, tag);
     }
   }
 }
@@ -749,16 +1107,18 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-size_t state_bf16_smem_bytes() { return st::kSmemBytes; }
-size_t out_bf16_smem_bytes() { return ot::kSmemBytes; }
+size_t state_bf16_smem_bytes() { return kStateSmem; }
+size_t out_bf16_smem_bytes() { return kOutSmem; }
 size_t state_f32_smem_bytes() { return kStateF32Smem; }
 size_t out_f32_smem_bytes() { return kOutF32Smem; }
 
 cudaError_t set_kernel_attributes() {
   cudaError_t e;
-  e = cudaFuncSetAttribute(state_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, st::kSmemBytes);
+  e = cudaFuncSetAttribute(state_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(out_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ot::kSmemBytes);
+  e = cudaFuncSetAttribute(fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fu::kSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(out_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateF32Smem);
   if (e != cudaSuccess) return e;
@@ -767,24 +1127,46 @@ cudaError_t set_kernel_attributes() {
 
 cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,
                               uint32_t* status, cudaStream_t s) {
-  return launch_pdl(state_bf16_kernel, dim3(g.G), dim3(kThreads), st::kSmemBytes, s, k.main, k.last, v.main, v.last,
+  return launch_pdl(state_bf16_kernel, dim3(g.G), dim3(kThreads), kStateSmem, s, k.main, k.last, v.main, v.last,
                     g, partials, segcta, status);
 }
 
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles, float eps,
                             uint32_t* status, cudaStream_t s) {
-  return launch_pdl(out_bf16_kernel, dim3(g.G), dim3(kThreads), ot::kSmemBytes, s, q.main, q.last, o.main, o.last,
+  return launch_pdl(out_bf16_kernel, dim3(g.G), dim3(kThreads), kOutSmem, s, q.main, q.last, o.main, o.last,
                     g, static_cast<const uint8_t*>(ptiles), eps, status);
 }
 
-cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in, float* S_out,
-                        float* z_out, void* ptiles_bf16, float* p32, cudaStream_t s) {
+cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
+                              const Geom& g, float* partials, int2* segcta, uint64_t* flags, void* ptiles,
+                              const float* S_in, const float* z_in, float* S_out, float* z_out, float eps,
+                              uint32_t* status, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g.G);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = fu::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barriers can complete
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fused_bf16_kernel, k.main, k.last, v.main, v.last, q.main, q.last, o.main, o.last,
+                            g, partials, segcta, flags, flags + g.nslots, static_cast<uint8_t*>(ptiles), S_in, z_in,
+                            S_out, z_out, eps, status);
+}
+
+cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
+                        float* S_out, float* z_out, void* ptiles_bf16, float* p32, cudaStream_t s) {
+  // ng warps share the blocks of one row; R rows per block so that a block has up to 16 warps
   int ng = (g.nblk + kScanReg - 1) / kScanReg;
   if (ng > kScanMaxWarps) ng = kScanMaxWarps;
   if (ng < 1) ng = 1;
-  return launch_pdl(scan_kernel, dim3(g.BH, kPTileRows), dim3(32 * ng), (ng + 1) * 32 * sizeof(float4), s,
-                    partials, segcta, g, S_in, z_in, S_out,
-                    z_out, static_cast<uint8_t*>(ptiles_bf16), p32);
+  int R = 16;
+  while (R > 1 && (R * ng > 16 || kPTileRows % R != 0)) R >>= 1;
+  const size_t smem = static_cast<size_t>(R) * (ng + 1) * 32 * sizeof(float4);
+  return launch_pdl(scan_kernel, dim3(g.BH, kPTileRows / R), dim3(32 * ng * R), smem, s, partials, segcta, g, S_in,
+                    z_in, S_out, z_out, static_cast<uint8_t*>(ptiles_bf16), p32, ng);
 }
 
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,

@@ -67,8 +67,10 @@ extern "C" sv_status sv_cache_step_noalloc(const void* q, const void* k, const v
     }
     ws = g_scratch_addr[dev];
   }
-  // the 256-byte header (status word) must start at zero; the rest is fully rewritten by each call
-  if (cudaMemsetAsync(ws, 0, sv::kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // the status word must start at zero; the launch sequence number and the flags behind it keep
+  // their values from call to call (the array starts zeroed when the library loads), and the rest is
+  // fully rewritten by each call
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return sv::set_last_error(SV_ERR_CUDA, "sv_cache_step_noalloc: clearing the scratch header failed");
   return sv_cache_step(q, k, v, o, B, H, N, D, dt, eps, S, z, commit, ws, kNoAllocScratchBytes, stream);
 }
