@@ -195,6 +195,24 @@ def _traffic(kernel: str):
     return None
 
 
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings over all ranks (no-op for one rank). Works on any
+    torch.distributed backend: CUDA tensors for NCCL, CPU tensors for gloo."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_value(world: int, tokheads_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the units every rank processed divided by the slowest rank's time."""
+    return world * tokheads_per_rank * steps / (max_ms / 1e3)
+
+
 def run_ours(args, rank: int, world: int):
     import torch
     import torch.distributed as dist
@@ -260,15 +278,12 @@ def run_ours(args, rank: int, world: int):
     st_ms = sum(r[0].elapsed_time(r[1]) for r in evs) / n_prof
     sc_ms = sum(r[1].elapsed_time(r[2]) for r in evs) / n_prof
     ou_ms = sum(r[2].elapsed_time(r[3]) for r in evs) / n_prof
-    if world > 1:
-        t = torch.tensor([ms, st_ms, sc_ms, ou_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, st_ms, sc_ms, ou_ms = t.tolist()
+    ms, st_ms, sc_ms, ou_ms = max_over_ranks([ms, st_ms, sc_ms, ou_ms], world, dev)
     if ws.status() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
 
     tokheads = B * H * N
-    value = world * tokheads * args.steps / (ms / 1e3)
+    value = aggregate_value(world, tokheads, args.steps, ms)
     ms_step = ms / args.steps
 
     # end to end through the public API: pinned host inputs -> device -> call -> o back to host
@@ -295,11 +310,7 @@ def run_ours(args, rank: int, world: int):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        ems = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = t.item()
+        ems = max_over_ranks([a.elapsed_time(b)], world, dev)[0]
         e2e = {"value": world * tokheads * n_e2e / (ems / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2,
                "steps": n_e2e, "ms_per_step": ems / n_e2e}
