@@ -24,5 +24,6 @@ from ._native import (  # noqa: F401
     sv_cache_step_noalloc,
     sv_linattn_fwd,
     sv_profile_events,
+    sv_selftest_wait_timeout,
     workspace_bytes,
 )

@@ -26,7 +26,7 @@ SV_OP_LINATTN_FWD, SV_OP_BLOCK_STATE_UPDATE, SV_OP_BLOCK_CAUSAL_ATTN, SV_OP_CACH
 EXPORTS = (
     "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_linattn_fwd",
     "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_cache_step_noalloc",
-    "sv_profile_events", "sv_last_error", "sv_version",
+    "sv_profile_events", "sv_last_error", "sv_selftest_wait_timeout", "sv_version",
 )
 
 
@@ -70,6 +70,8 @@ def load() -> ctypes.CDLL:
         lib.sv_profile_events.restype = i
         lib.sv_last_error.argtypes = []
         lib.sv_last_error.restype = ctypes.c_char_p
+        lib.sv_selftest_wait_timeout.argtypes = [vp, sz, vp]
+        lib.sv_selftest_wait_timeout.restype = i
         lib.sv_version.argtypes = []
         lib.sv_version.restype = i
         _lib = lib
@@ -139,6 +141,12 @@ class Workspace:
         if st not in (SV_OK, SV_ERR_TIMEOUT):
             _check(st)
         return int(code.value)
+
+
+def sv_selftest_wait_timeout(ws: Workspace, stream=None):
+    """Launch the bounded-wait self-test on `ws` (its status word is raised about 2 s later; read it
+    with ws.status())."""
+    _check(load().sv_selftest_wait_timeout(ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def make_workspace(op: int, q_like: torch.Tensor, block_len: int | None = None, stream=None) -> Workspace:

@@ -96,6 +96,24 @@ SV_HD int seg_ntiles(int seg, const Geom& q) {
   return (b == q.nblk - 1) ? q.tpl : q.tpb;
 }
 
+// The combine of head h (one block per head) is shared by the CTAs [ga, gb]: those whose tile
+// range starts inside the head, or, when none does, the CTA holding the head's first tile. Each
+// CTA then combines one head, apart from heads shorter than a CTA's range.
+struct CombineRange {
+  int g0, g1;  // CTAs covering the head (their slots g + h hold its partial states)
+  int ga, gb;  // CTAs sharing its combine
+};
+SV_HD CombineRange combine_range(int h, const Geom& geo) {
+  const long long f = seg_first_tile(h, geo);
+  CombineRange r;
+  r.g0 = cta_of_tile(f, geo);
+  r.g1 = cta_of_tile(f + seg_ntiles(h, geo) - 1, geo);
+  r.ga = tile_begin(r.g0, geo) == f ? r.g0 : r.g0 + 1;
+  r.gb = r.g1;
+  if (r.ga > r.gb) r.ga = r.gb = r.g0;
+  return r;
+}
+
 // Host-side construction. Returns false when the sizes are out of range.
 inline bool make_geom(Geom& q, int B, int H, int N, int D, int block_len, int sm_count) {
   if (B <= 0 || H <= 0 || N <= 0 || D <= 0 || block_len <= 0 || sm_count <= 0) return false;

@@ -14,9 +14,13 @@
 //   3. out_bf16_kernel    : per tile, TMA Q -> ReLU(Q) in shared memory -> tcgen05.mma
 //      ReLU(Q) x [P | z]^T into TMEM; the epilogue divides numerator by (denominator + eps),
 //      converts to bf16 and TMA-stores the tile.
+// When every head is a single block (bidirectional layer, streaming step), fused_bf16_kernel runs
+// the three steps in one launch of co-resident CTAs: the state roles, a per-head combine shared by
+// the CTAs that cover the head (synchronised through release/acquire flags), then the output roles.
 // The fp32 I/O path runs the same three steps with SIMT fp32 kernels.
 #include <cuda_bf16.h>
 
+#include <cstdlib>
 #include <utility>
 
 #include "sv_internal.h"
@@ -78,6 +82,11 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // ---- flags between CTAs of the single-launch kernel (release / acquire at GPU scope) ----
 __device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel_u32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
   uint64_t v;
@@ -315,7 +324,8 @@ constexpr int kQBytes = 2 * kAtomBytes;             // Q tile: 128 tokens x 128 
 constexpr int kBOff = kStages * kQBytes;            // two prefix tiles (double-buffered)
 constexpr int kBAtomBytes = kPTileRows * 128;       // 144 rows x 128 B
 constexpr int kOOff = kBOff + 2 * kPTileBytes;      // output staging, one 8 KB slice per warp
-constexpr int kOWarpBytes = 2 * 32 * 128;
+constexpr int kOWarpBytes = 2 * 32 * 128;      // two 4 KB atoms: output columns 0..63 and 64..127
+constexpr int kAtomBytesO = 32 * 128;
 constexpr int kRegionBytes = kOOff + 4 * kOWarpBytes;
 constexpr int kNumBars = 18;
 static_assert(kBOff % 1024 == 0 && kOOff % 1024 == 0 && kBAtomBytes % 1024 == 0, "1024-B atoms");
@@ -333,7 +343,10 @@ struct Bars {
 __device__ __forceinline__ Bars bars_at(uint64_t* p) {
   return Bars{p, p + 3, p + 6, p + 9, p + 11, p + 13, p + 15, p + 17};
 }
-__device__ __forceinline__ void init_bars(const Bars& b) {
+// The epilogue of a tile runs on 4 warps per 64 output columns: 8 warps for D > 64, else 4.
+__device__ __forceinline__ int epi_warps(bool two_atoms) { return two_atoms ? 8 : 4; }
+
+__device__ __forceinline__ void init_bars(const Bars& b, bool two_atoms) {
   for (int i = 0; i < kStages; ++i) {
     mbar_init(&b.qfull[i], 1);
     mbar_init(&b.qrelu[i], 4);
@@ -343,7 +356,7 @@ __device__ __forceinline__ void init_bars(const Bars& b) {
     mbar_init(&b.bfull[a], 1);
     mbar_init(&b.bempty[a], 1);
     mbar_init(&b.accf[a], 1);
-    mbar_init(&b.acce[a], 4);
+    mbar_init(&b.acce[a], epi_warps(two_atoms));
   }
   mbar_init(b.done, 1);
 }
@@ -373,7 +386,9 @@ __device__ int prefill(uint8_t* smem, const Bars& b, const Maps4& m, const Geom&
 // The rest of the producer: prefix tiles (read only once the prefix is complete) and the Q tiles
 // after the prefilled ones.
 // With `combined` (single-launch kernel, one block per head), a head's prefix tile is loaded only
-// once every CTA covering the head has published its share of the combine (value `tag`).
+// once every CTA sharing the head's combine has published its rows (value `tag`). With ptiles ==
+// nullptr the prefix tiles are already in shared memory (buffer j & 1 for the j-th segment) and
+// are only signalled to the MMA warp.
 __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb, long long te,
                         int pre, bool two_atoms, const uint8_t* __restrict__ ptiles, const uint64_t* combined,
                         uint64_t tag, uint32_t* status) {
@@ -382,12 +397,15 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
   bool ok = true;
   for (long long t = tb; t < te && ok; ++t, ++k) {
     const TileCoord c = tile_coord(t, geo);
-    if (c.seg != prev) {
+    if (c.seg != prev && ptiles == nullptr) {  // the caller already placed the tile in buffer j & 1
+      mbar_arrive(&b.bfull[j & 1]);
+      ++j;
+      prev = c.seg;
+    } else if (c.seg != prev) {
       const int bb = j & 1;
       if (combined != nullptr) {
-        const long long f = seg_first_tile(c.seg, geo);
-        const int g0 = cta_of_tile(f, geo), g1 = cta_of_tile(f + seg_ntiles(c.seg, geo) - 1, geo);
-        if (!wait_flags(combined, g0 + c.seg, g1 + c.seg, tag, status, 0x2200u)) break;
+        const CombineRange cr = combine_range(c.seg, geo);
+        if (!wait_flags(combined, cr.ga + c.seg, cr.gb + c.seg, tag, status, 0x2200u)) break;
         fence_proxy_async_global();  // prefix tile written by other CTAs -> bulk copy below
       }
       if (!mbar_wait(&b.bempty[bb], ((j >> 1) & 1) ^ 1, status, 0x1100u | bb)) break;
@@ -406,21 +424,6 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
   for (int i = (k > kStages ? k - kStages : 0); i < (k > pre ? k : pre); ++i)
     mbar_wait(&b.qfull[i % kStages], (i / kStages) & 1, status, 0x1180u);
   for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&b.bfull[i & 1], (i >> 1) & 1, status, 0x1190u);
-}
-
-__device__ void relu_role(uint8_t* smem, const Bars& b, long long tb, long long te, bool two_atoms, int r, int lane,
-                          uint32_t* status) {
-  const int nchunks = (two_atoms ? kQBytes : kAtomBytes) / 16;
-  int k = 0;
-  for (long long t = tb; t < te; ++t, ++k) {
-    const int s = k % kStages;
-    bool ok = mbar_wait(&b.qfull[s], (k / kStages) & 1, status, 0x1200u | s);
-    if (!warp_all(ok)) break;
-    relu_tile_inplace(smem + s * kQBytes, nchunks, r);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&b.qrelu[s]);
-  }
 }
 
 __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, bool two_atoms,
@@ -460,72 +463,96 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long lon
   mbar_wait(b.done, 0, status, 0x13F0u);
 }
 
-// Epilogue: warp w owns tokens 32w..32w+31 of the tile (TMEM lanes); numerator columns times
-// 1 / (denominator + eps), bf16, swizzled staging, TMA store clipped to the block.
-__device__ void epilogue_role(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
-                              long long te, bool two_atoms, uint32_t tmem, int warp, int lane, float eps,
-                              uint32_t* status) {
-  uint8_t* ob = smem + kOOff + warp * kOWarpBytes;
-  const int ncc = two_atoms ? 4 : 2;
-  int k = 0;
-  for (long long t = tb; t < te; ++t, ++k) {
-    const TileCoord c = tile_coord(t, geo);
-    const int a = k & 1;
-    bool ok = mbar_wait(&b.accf[a], (k >> 1) & 1, status, 0x1400u | a);
-    if (!warp_all(ok)) break;
-    tc_fence_after();
-    const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(a * 256);
-    // two halves of 64 columns, each read with one wait (the register budget holds 64 values)
-    uint32_t dr;
-    tmem_ld_x1(ta + kZRow, dr);
-    float inv = 0.f;
-    for (int h = 0; h < 2; ++h) {
-      if (2 * h >= ncc) break;
-      uint32_t rr[2][32];
-      tmem_ld_x32(ta + h * 64, rr[0]);
-      tmem_ld_x32(ta + h * 64 + 32, rr[1]);
-      tmem_wait_ld();
-      if (h == 0) {
-        inv = __frcp_rn(__uint_as_float(dr) + eps);
-        if (lane == 0) bulk_wait_read_all();  // the previous store has finished reading the slice
-        __syncwarp();
-      }
-      if (2 * h + 2 >= ncc) {  // last half read: the accumulator is free
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b.acce[a]);
-      }
+// ReLU of Q tile k (stage k % kStages) in place; returns false if the grid failed.
+__device__ __forceinline__ bool relu_q(uint8_t* smem, const Bars& b, long long k, bool two_atoms, int r, int lane,
+                                       uint32_t* status) {
+  const int s = static_cast<int>(k % kStages);
+  const bool ok = mbar_wait(&b.qfull[s], static_cast<uint32_t>((k / kStages) & 1), status, 0x1200u | s);
+  if (!warp_all(ok)) return false;
+  relu_tile_inplace(smem + s * kQBytes, (two_atoms ? kQBytes : kAtomBytes) / 16, r);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&b.qrelu[s]);
+  return true;
+}
+
+// Epilogue of tile k for one warp: TMEM lanes 32q..32q+31 (q = warp % 4, tokens of the tile) and
+// output columns 64h..64h+63; numerator times 1 / (denominator + eps), bf16, into this warp's
+// swizzled 4 KB staging atom, then a TMA store clipped to the block.
+__device__ __forceinline__ bool epilogue_tile(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo,
+                                              long long t, long long k, uint32_t tmem, int q, int h, int lane,
+                                              float eps, uint32_t* status) {
+  const TileCoord c = tile_coord(t, geo);
+  const int a = static_cast<int>(k & 1);
+  const bool ok = mbar_wait(&b.accf[a], static_cast<uint32_t>((k >> 1) & 1), status, 0x1400u | a);
+  if (!warp_all(ok)) return false;
+  tc_fence_after();
+  const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
+  uint32_t dr;
+  uint32_t rr[2][32];
+  tmem_ld_x1(ta + kZRow, dr);
+  tmem_ld_x32(ta + h * 64, rr[0]);
+  tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+  tmem_wait_ld();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&b.acce[a]);  // the values are in registers: the accumulator is free
+  const float inv = __frcp_rn(__uint_as_float(dr) + eps);
+  uint8_t* ob = smem + kOOff + q * kOWarpBytes + h * kAtomBytesO;
+  if (lane == 0) bulk_wait_read_all();  // this warp's previous store has finished reading the atom
+  __syncwarp();
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+  for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 0]) * inv, __uint_as_float(rr[cc][8 * mm + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 2]) * inv, __uint_as_float(rr[cc][8 * mm + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 4]) * inv, __uint_as_float(rr[cc][8 * mm + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 6]) * inv, __uint_as_float(rr[cc][8 * mm + 7]) * inv);
-          const int chunk = (2 * h + cc) * 4 + mm;  // 16-byte chunk of the 256-byte output row
-          uint8_t* dst = ob + (chunk >> 3) * 4096 + lane * 128 + (((chunk & 7) ^ (lane & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = w;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      const int blen = (c.blk == geo.nblk - 1) ? geo.Llast : geo.L;
-      const int row0 = c.tok0 + warp * 32;
-      if (row0 < blen) {
-        const bool lst = use_last_map(c, geo);
-        const CUtensorMap* mo = lst ? m.b_last : m.b_main;
-        const int cb = lst ? 0 : c.blk;
-        tma_store_4d(mo, ob, 0, row0, cb, c.bh);
-        if (two_atoms) tma_store_4d(mo, ob + 4096, 64, row0, cb, c.bh);
-        bulk_commit();
-      }
+    for (int mm = 0; mm < 4; ++mm) {
+      uint4 w;
+      w.x = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 0]) * inv, __uint_as_float(rr[cc][8 * mm + 1]) * inv);
+      w.y = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 2]) * inv, __uint_as_float(rr[cc][8 * mm + 3]) * inv);
+      w.z = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 4]) * inv, __uint_as_float(rr[cc][8 * mm + 5]) * inv);
+      w.w = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 6]) * inv, __uint_as_float(rr[cc][8 * mm + 7]) * inv);
+      const int chunk = cc * 4 + mm;  // 16-byte chunk of the 128-byte row of this atom
+      *reinterpret_cast<uint4*>(ob + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = w;
     }
   }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    const int blen = (c.blk == geo.nblk - 1) ? geo.Llast : geo.L;
+    const int row0 = c.tok0 + q * 32;
+    if (row0 < blen) {
+      const bool lst = use_last_map(c, geo);
+      tma_store_4d(lst ? m.b_last : m.b_main, ob, h * 64, row0, lst ? 0 : c.blk, c.bh);
+      bulk_commit();
+    }
+  }
+  return true;
+}
+
+// Warps 0-3: epilogue of output columns 0..63 of every tile.
+__device__ void epilogue_role(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
+                              long long te, uint32_t tmem, int warp, int lane, float eps, uint32_t* status) {
+  long long k = 0;
+  for (long long t = tb; t < te; ++t, ++k)
+    if (!epilogue_tile(smem, b, m, geo, t, k, tmem, warp & 3, 0, lane, eps, status)) break;
   if (lane == 0) bulk_wait_all();
+}
+
+// Warps 4-7: ReLU of the Q tiles, running up to kStages tiles ahead, and (D > 64) the epilogue of
+// output columns 64..127. Tile k + kStages is ReLU'd after the epilogue of tile k: its stage was
+// freed by the MMAs of tile k, which the epilogue has waited for, so the order cannot deadlock.
+__device__ void relu_epi_role(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
+                              long long te, bool two_atoms, uint32_t tmem, int warp, int lane, float eps,
+                              uint32_t* status) {
+  const int r = static_cast<int>(threadIdx.x) - 128;
+  const long long n = te - tb;
+  long long kr = 0;
+  bool ok = true;
+  for (; kr < n && kr < kStages && ok; ++kr) ok = relu_q(smem, b, kr, two_atoms, r, lane, status);
+  for (long long k = 0; k < n && ok; ++k) {
+    if (two_atoms) ok = epilogue_tile(smem, b, m, geo, tb + k, k, tmem, warp & 3, 1, lane, eps, status);
+    if (ok && kr < n) ok = relu_q(smem, b, kr++, two_atoms, r, lane, status);
+  }
+  if (two_atoms && lane == 0) bulk_wait_all();
 }
 }  // namespace ot
 
@@ -615,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool two_atoms = geo.D > 64;
   const Maps4 m{&q_main, &q_last, &o_main, &o_last};
   if (threadIdx.x == 0) {
-    ot::init_bars(b);
+    ot::init_bars(b, two_atoms);
     fence_mbar_init();
   }
   if (warp == kWarpProducer && lane == 0) prefetch_maps(m);
@@ -628,11 +655,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ot::produce(smem, b, m, geo, tb, te, pre, two_atoms, ptiles, nullptr, 0, status);
     }
   } else if (warp >= 4 && warp < 8) {
-    ot::relu_role(smem, b, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+    ot::relu_epi_role(smem, b, m, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
   } else if (warp == kWarpMma) {
     if (lane == 0) ot::mma_role(smem, b, geo, tb, te, two_atoms, tmem, status);
   } else {
-    ot::epilogue_role(smem, b, m, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
+    ot::epilogue_role(smem, b, m, geo, tb, te, tmem, warp, lane, eps, status);
   }
   persistent_teardown(tmem, warp);
 }
@@ -774,92 +801,150 @@ __global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ pa
 // ------------------------------------------------------------------------------------------
 // 4. one launch for one-block problems (bidirectional forward, streaming cache step)
 // ------------------------------------------------------------------------------------------
-// State reduction -> combine -> output in one cooperative launch (every CTA resident, one per SM).
+// State reduction -> combine -> output in one launch (every CTA resident, one per SM).
 // Each CTA reduces and then outputs the same contiguous tile range; heads are synchronised one by
 // one instead of with grid-wide barriers: a CTA publishes each partial slot it flushes; the CTAs
-// covering a head split that head's combine once all its slots are published, and publish their
-// share; a head's output starts once its combine is complete. Flags carry the workspace's launch
-// sequence number (header bytes 8..15, advanced by the last CTA to exit), so nothing needs resetting.
-// The stage memory of the reduction is reused by the output, whose first Q tiles load before the
-// combine.
+// whose range starts inside a head split that head's combine once all its slots are published
+// (reading their share of the incoming cache while they wait, writing the outgoing cache after
+// publishing), and publish their share; a head's output starts once its combine is complete.
+// Flags carry the workspace's launch sequence number (header bytes 8..15, advanced by the last CTA
+// to read it), so nothing needs resetting. The stage memory of the reduction is reused by the output,
+// whose first Q tiles load while the combine runs.
 namespace fu {
 constexpr int kRegion = (st::kRegionBytes > ot::kRegionBytes) ? st::kRegionBytes : ot::kRegionBytes;
 constexpr int kSmem = kRegion + 512 + 1024;
 // shared memory free during the combine (between the prefilled Q stages and the output staging):
 // the cache transpose of up to 128 rows x 129 floats
 constexpr int kScratchOff = ot::kBOff;
-static_assert(kScratchOff + 128 * 129 * 4 <= ot::kOOff, "combine scratch overlaps the output staging");
+constexpr int kScratchZOff = kScratchOff + 128 * 129 * 4;  // z row of the share (128 floats)
+static_assert(kScratchZOff + 128 * 4 <= ot::kOOff, "combine scratch overlaps the output staging");
 }  // namespace fu
 
-// This CTA's share of head bh's combine: rows [r0, r1) of the prefix tile (row e < 128: value
-// feature e of S; row 128: z; rows 129..143: zero), each row = S_in/z_in + the head's partial slots
-// of CTAs g0..g1, written as the bf16 B operand of the output GEMM and, when asked, to the cache.
-// The cache is [d][e] (key feature major) while a prefix row is one value feature e, so S_in and
-// S_out go through a shared-memory transpose `sS` to keep the global accesses coalesced.
-__device__ void combine_rows(const Geom& geo, const float* __restrict__ partials, int g0, int g1, const float* S_in,
-                             const float* z_in, float* S_out, float* z_out, uint8_t* __restrict__ ptiles, int bh,
-                             int r0, int r1, float* sS) {
-  const int D = geo.D;
-  const int e_hi = (r1 < D ? r1 : D);          // S rows of the share: [r0, e_hi)
-  const int ns = e_hi > r0 ? e_hi - r0 : 0;
-  const int ld = D + 1;                         // padded row of sS
-  if (S_in != nullptr && ns > 0) {
-    for (int i = threadIdx.x; i < D * ns; i += kThreads) {
-      const int d = i / ns, j = i - d * ns;     // consecutive threads: consecutive e of one key row d
-      sS[j * ld + d] = S_in[(static_cast<size_t>(bh) * D + d) * D + r0 + j];
+// Rows [r0, r1) of head bh's prefix tile (row e < 128: value feature e of S; row 128: z; rows
+// 129..143: zero). The cache is [d][e] (key feature major) while a prefix row is one value feature
+// e, so S_in and S_out go through the shared-memory transpose sS ([row - r0][d], padded rows) and
+// the global side stays coalesced. Row kZRow's z values go through sZ.
+__device__ __forceinline__ int cache_rows(const Geom& geo, int r0, int r1) {
+  const int e_hi = (r1 < geo.D ? r1 : geo.D);
+  return e_hi > r0 ? e_hi - r0 : 0;
+}
+
+// Step 1 (independent of the other CTAs): the incoming cache rows of the share into sS / sZ.
+// Threads tid = 0..nthr-1 of the caller share the work.
+__device__ void combine_load_cache(const Geom& geo, const float* S_in, const float* z_in, int bh, int r0, int r1,
+                                   float* sS, float* sZ, int tid, int nthr) {
+  const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1);
+  if (S_in != nullptr) {
+    // consecutive threads read consecutive e of one key row d; 8 loads per thread in flight
+    for (int i0 = tid; i0 < D * ns; i0 += 8 * nthr) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * nthr;
+        const int d = i / ns, j = i - d * ns;
+        v[u] = i < D * ns ? __ldcg(S_in + (static_cast<size_t>(bh) * D + d) * D + r0 + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * nthr;
+        const int d = i / ns, j = i - d * ns;
+        if (i < D * ns) sS[j * ld + d] = v[u];
+      }
     }
   }
-  __syncthreads();
-  for (int it = r0 * 32 + static_cast<int>(threadIdx.x); it < r1 * 32; it += kThreads) {
-    const int e = it >> 5;
-    const int d0 = (it & 31) * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (e < kPartRows) {
-      for (int gg = g0; gg <= g1; ++gg) {
-        const float4 p = *reinterpret_cast<const float4*>(
-            partials + (static_cast<size_t>(gg + bh) * kPartRows + e) * kDPad + d0);
-        acc[0] += p.x;
-        acc[1] += p.y;
-        acc[2] += p.z;
-        acc[3] += p.w;
+  if (z_in != nullptr && r0 <= kZRow && kZRow < r1)
+    for (int d = tid; d < D; d += nthr) sZ[d] = __ldcg(z_in + static_cast<size_t>(bh) * D + d);
+}
+
+// Step 2 (once the head's partial slots exist): each row = cache + the slots of CTAs g0..g1 in
+// ascending order, written as the bf16 B operand of the output GEMM; the sums replace the cache
+// values in sS / sZ for step 3. Each thread takes two (row, quad) items per pass and keeps up to 8
+// slots of each in flight at once; the order of the additions does not depend on the unrolling.
+__device__ void combine_sum(const Geom& geo, const float* __restrict__ partials, int g0, int g1, bool has_S,
+                            bool has_z, uint8_t* __restrict__ ptiles, int bh, int r0, int r1, float* sS, float* sZ) {
+  const int D = geo.D, ld = D + 1;
+  for (int base = r0 * 32 + static_cast<int>(threadIdx.x); base < r1 * 32; base += 2 * kThreads) {
+    int es[2], ds[2];
+    bool vs[2];
+    float acc[2][4];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int it = base + x * kThreads;
+      es[x] = it >> 5;
+      ds[x] = (it & 31) * 4;
+      vs[x] = it < r1 * 32 && es[x] < kPartRows;
+      acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
+    }
+    for (int gb = g0; gb <= g1; gb += 8) {
+      float4 p[2][8];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          p[x][u] = (vs[x] && gb + u <= g1)
+                        ? __ldcg(reinterpret_cast<const float4*>(
+                              partials + (static_cast<size_t>(gb + u + bh) * kPartRows + es[x]) * kDPad + ds[x]))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (gb + u <= g1) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            acc[x][0] += p[x][u].x;
+            acc[x][1] += p[x][u].y;
+            acc[x][2] += p[x][u].z;
+            acc[x][3] += p[x][u].w;
+          }
+        }
       }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int it = base + x * kThreads;
+      if (it >= r1 * 32) break;
+      const int e = es[x], d0 = ds[x];
+      float* a = acc[x];
       if (e < D) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (d0 + u < D) {
-            if (S_in != nullptr) acc[u] += sS[(e - r0) * ld + d0 + u];
-            if (S_out != nullptr) sS[(e - r0) * ld + d0 + u] = acc[u];
+            float* c = &sS[(e - r0) * ld + d0 + u];
+            if (has_S) a[u] += *c;
+            *c = a[u];
           }
         }
-      }
-      if (e == kZRow) {
+      } else if (e == kZRow) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (d0 + u < D) {
-            if (z_in != nullptr) acc[u] += z_in[static_cast<size_t>(bh) * D + d0 + u];
+            if (has_z) a[u] += sZ[d0 + u];
+            sZ[d0 + u] = a[u];
           }
         }
-        if (z_out != nullptr) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (d0 + u < D) z_out[static_cast<size_t>(bh) * D + d0 + u] = acc[u];
-        }
       }
+      uint2 w;
+      w.x = pack_bf16x2(a[0], a[1]);
+      w.y = pack_bf16x2(a[2], a[3]);
+      const size_t off = static_cast<size_t>(bh) * kPTileBytes + (d0 >> 6) * (kPTileRows * 128) + e * 128 +
+                         ((((d0 & 63) >> 3) ^ (e & 7)) << 4) + (d0 & 7) * 2;
+      *reinterpret_cast<uint2*>(ptiles + off) = w;
     }
-    uint2 w;
-    w.x = pack_bf16x2(acc[0], acc[1]);
-    w.y = pack_bf16x2(acc[2], acc[3]);
-    const size_t off = static_cast<size_t>(bh) * kPTileBytes + (d0 >> 6) * (kPTileRows * 128) + e * 128 +
-                       ((((d0 & 63) >> 3) ^ (e & 7)) << 4) + (d0 & 7) * 2;
-    *reinterpret_cast<uint2*>(ptiles + off) = w;
   }
-  __syncthreads();
-  if (S_out != nullptr && ns > 0) {
+}
+
+// Step 3 (after the prefix rows are published; nothing in this launch reads the outgoing cache):
+// the share's rows of the outgoing cache from sS / sZ.
+__device__ void combine_store_cache(const Geom& geo, float* S_out, float* z_out, int bh, int r0, int r1,
+                                    const float* sS, const float* sZ) {
+  const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1);
+  if (S_out != nullptr) {
     for (int i = threadIdx.x; i < D * ns; i += kThreads) {
       const int d = i / ns, j = i - d * ns;
       S_out[(static_cast<size_t>(bh) * D + d) * D + r0 + j] = sS[j * ld + d];
     }
   }
+  if (z_out != nullptr && r0 <= kZRow && kZRow < r1)
+    for (int d = threadIdx.x; d < D; d += kThreads) z_out[static_cast<size_t>(bh) * D + d] = sZ[d];
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -881,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* flushed = barmem + st::kNumBars + ot::kNumBars;  // epilogue warps finished a slot (count 4)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flushed + 1);
   uint64_t* seqp = reinterpret_cast<uint64_t*>(status + 2);  // header bytes 8..15: launch sequence number
-  uint32_t* gexit = status + 4;                              // header bytes 16..19: CTAs that finished
+  uint32_t* gstart = status + 4;                             // header bytes 16..19: CTAs that read the tag
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -893,11 +978,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Maps4 mqo{&q_main, &q_last, &o_main, &o_last};
   if (threadIdx.x == 0) {
     st::init_bars(sb);
-    ot::init_bars(ob);
+    ot::init_bars(ob, two_atoms);
     mbar_init(flushed, 4);
     fence_mbar_init();
-    s_ok = 1;
-    s_tag = ld_acquire_u64(seqp) + 1;
   }
   st::init_smem(smem, two_atoms, kThreads);
   if (warp == kWarpProducer && lane == 0) {
@@ -905,15 +988,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_maps(mqo);
   }
   const uint32_t tmem = persistent_setup(tmem_slot, warp);
-  const uint64_t tag = s_tag;
+  // Up to here only this CTA's shared memory and TMEM were touched, so this part overlaps the
+  // previous kernel in the stream (programmatic dependent launch). That kernel may still write
+  // q, k, v, the cache or this workspace: wait for it to complete before any global access.
+  griddep_wait();
+  // Thread 0 (epilogue warp 0) is the only user of the launch tag before phase 2: it reads the tag
+  // here, off the other roles' path, and shares it through s_tag with phase 2 and 3.
+  uint64_t tag = 0;
+  if (threadIdx.x == 0) {
+    s_ok = 1;
+    tag = ld_acquire_u64(seqp) + 1;
+    s_tag = tag;
+    // The last CTA to read the sequence number advances it for the next launch on this workspace:
+    // every CTA has read it by then (acq_rel orders each CTA's read before its increment), and the
+    // next launch reads it only after this one has completed.
+    if (atom_add_acq_rel_u32(gstart, 1u) == static_cast<uint32_t>(G - 1)) {
+      *gstart = 0u;
+      st_release_u64(seqp, tag);
+    }
+    griddep_launch_dependents();  // the next launch may now set up on SMs as they free up
+  }
 
-  // phase 1: block states of this CTA's tiles; the producer then fills the first Q stages
+  // phase 1: block states of this CTA's tiles
   int pre = 0;
   if (warp == kWarpProducer) {
-    if (lane == 0) {
-      st::produce(smem, sb, mkv, geo, tb, te, two_atoms, false, status);
-      pre = ot::prefill(smem, ob, mqo, geo, tb, te, two_atoms);
-    }
+    if (lane == 0) st::produce(smem, sb, mkv, geo, tb, te, two_atoms, false, status);
   } else if (warp >= 4 && warp < 8) {
     st::relu_role(smem, sb, tb, te, two_atoms, threadIdx.x - 128, lane, status);
   } else if (warp == kWarpMma) {
@@ -923,25 +1022,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  tag = s_tag;
 
-  // phase 2: this CTA's share of the combine of each head it covers, once all the head's slots exist
+  // phase 2: the Q stages fill (Q does not depend on the state, and the stages are free once the
+  // state MMAs retired) while the CTA takes its share of the combine of its head(s): whole prefix
+  // rows, so each cache element belongs to exactly one CTA.
+  if (warp == kWarpProducer && lane == 0) pre = ot::prefill(smem, ob, mqo, geo, tb, te, two_atoms);
+  float* sS = reinterpret_cast<float*>(smem + fu::kScratchOff);
+  float* sZ = reinterpret_cast<float*>(smem + fu::kScratchZOff);
   const int h0 = tile_coord(tb, geo).seg;
   const int h1 = tile_coord(te - 1, geo).seg;
   for (int h = h0; h <= h1; ++h) {
-    const long long f = seg_first_tile(h, geo);
-    const int g0 = cta_of_tile(f, geo), g1 = cta_of_tile(f + seg_ntiles(h, geo) - 1, geo);
-    if (threadIdx.x == 0 && s_ok && !wait_flags(slot_ready, g0 + h, g1 + h, tag, status, 0x2000u)) s_ok = 0;
+    const CombineRange cr = combine_range(h, geo);
+    if (g < cr.ga || g > cr.gb) continue;
+    const int n = cr.gb - cr.ga + 1, idx = g - cr.ga;
+    const int r0 = idx * kPTileRows / n, r1 = (idx + 1) * kPTileRows / n;
+    combine_load_cache(geo, S_in, z_in, h, r0, r1, sS, sZ, threadIdx.x, kThreads);  // needs no other CTA
+    if (threadIdx.x == 0 && s_ok && !wait_flags(slot_ready, cr.g0 + h, cr.g1 + h, tag, status, 0x2000u)) s_ok = 0;
     __syncthreads();
-    if (s_ok) {  // whole rows per CTA, so each cache element belongs to exactly one CTA
-      const int n = g1 - g0 + 1, idx = g - g0;
-      combine_rows(geo, partials, g0, g1, S_in, z_in, S_out, z_out, ptiles, h, idx * kPTileRows / n,
-                   (idx + 1) * kPTileRows / n, reinterpret_cast<float*>(smem + fu::kScratchOff));
-    }
+    if (s_ok)
+      combine_sum(geo, partials, cr.g0, cr.g1, S_in != nullptr, z_in != nullptr, ptiles, h, r0, r1, sS, sZ);
     __syncthreads();
     if (threadIdx.x == 0 && s_ok) {
       __threadfence();
       st_release_u64(combined + g + h, tag);
     }
+    if (s_ok) combine_store_cache(geo, S_out, z_out, h, r0, r1, sS, sZ);
+    __syncthreads();
   }
   fence_proxy_async_smem();  // the combine scratch is next written by TMA copies (async proxy)
   __syncthreads();
@@ -952,24 +1059,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpProducer) {
       if (lane == 0) ot::produce(smem, ob, mqo, geo, tb, te, pre, two_atoms, ptiles, combined, tag, status);
     } else if (warp >= 4 && warp < 8) {
-      ot::relu_role(smem, ob, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+      ot::relu_epi_role(smem, ob, mqo, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
     } else if (warp == kWarpMma) {
       if (lane == 0) ot::mma_role(smem, ob, geo, tb, te, two_atoms, tmem, status);
     } else {
-      ot::epilogue_role(smem, ob, mqo, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
+      ot::epilogue_role(smem, ob, mqo, geo, tb, te, tmem, warp, lane, eps, status);
     }
   } else if (warp == kWarpProducer && lane == 0) {
     for (int i = 0; i < pre; ++i) mbar_wait(&ob.qfull[i], 0, status, 0x2180u);  // prefilled loads land
   }
   persistent_teardown(tmem, warp);
-  // the last CTA out advances the launch sequence number for the next launch on this workspace
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(gexit, 1u) == static_cast<uint32_t>(G - 1)) {
-      *gexit = 0u;
-      st_release_u64(seqp, tag);
-    }
-  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1146,9 +1245,27 @@ cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const Bloc
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = fu::kSmem;
   cfg.stream = s;
+  // The CTAs wait on one another (flags), so all of them must be resident at once: the grid has at
+  // most one CTA per SM and each SM fits exactly one (shared memory, TMEM), so on an otherwise idle
+  // device every CTA is placed. The launch uses programmatic stream serialization: each CTA sets up
+  // while the previous kernel drains and waits (griddepcontrol.wait) before any global access.
+  // A cooperative launch would also guarantee residency when other streams hold SMs, but the
+  // runtime then starts the grid only after the previous kernel has fully ended (measured: about
+  // 3 us later per launch). With SV_FUSED_COOPERATIVE=1 in the environment the launch is
+  // cooperative instead. Either way every wait is bounded: a CTA kept off the device for longer
+  // than the wait limit makes the call fail with the timeout status, never hang.
+  static const bool cooperative = [] {
+    const char* e = std::getenv("SV_FUSED_COOPERATIVE");
+    return e != nullptr && e[0] == '1';
+  }();
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barriers can complete
-  attr[0].val.cooperative = 1;
+  if (cooperative) {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, fused_bf16_kernel, k.main, k.last, v.main, v.last, q.main, q.last, o.main, o.last,

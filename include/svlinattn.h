@@ -35,6 +35,14 @@
  *    SV_ERR_CUDA. Device-side timeouts (SV_ERR_TIMEOUT) are reported by sv_device_status.
  *    sv_last_error() gives a message for the calling thread's last non-OK status.
  *  - NaN/Inf inputs propagate; nothing checks for them.
+ *  - Residency: with bf16 I/O and one block per head (sv_linattn_fwd, sv_cache_step and
+ *    sv_block_causal_attn with block_len >= N) the work runs as one launch whose CTAs (one per SM
+ *    at most) wait on one another, so they must all be resident together. On a device that other
+ *    streams do not occupy this always holds. The launch overlaps its setup with the previous
+ *    kernel (programmatic dependent launch); setting SV_FUSED_COOPERATIVE=1 in the environment
+ *    makes it a cooperative launch instead, which the runtime only starts once every CTA fits.
+ *    A CTA kept off the device for longer than the wait limit (2 s) makes the call report
+ *    SV_ERR_TIMEOUT through sv_device_status; it never hangs.
  */
 #ifndef SVLINATTN_H
 #define SVLINATTN_H
@@ -138,6 +146,16 @@ sv_status sv_profile_events(void* const* events, int n);
 const char* sv_last_error(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
+/* Failure-path self-test of the kernels' bounded waits; makes no GPU fault and leaves nothing in
+ * flight. Launches one CTA whose waiters block, through the same bounded-wait routine the pipeline
+ * kernels use, on an mbarrier phase that nothing completes. After the wait limit (about 2 s) the
+ * first waiter raises the status word of `ws` to 0x80000000 | 0x7E00 | warp and every waiter
+ * returns. Arguments: ws is a workspace (>= 256 bytes, 256-byte aligned, cleared by
+ * sv_workspace_init); stream as for every call. Returns SV_OK once the kernel is launched
+ * (SV_ERR_INVALID_ARG for a bad workspace, SV_ERR_CUDA if the launch fails); the expiry itself is
+ * read afterwards with sv_device_status, which then returns SV_ERR_TIMEOUT and clears the word. */
+sv_status sv_selftest_wait_timeout(void* ws, size_t ws_bytes, sv_stream_t stream);
+
 int sv_version(void);
 
 #ifdef __cplusplus

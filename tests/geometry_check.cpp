@@ -3,7 +3,9 @@
 //  - tiles never straddle blocks and cover every token exactly once,
 //  - the partial slot g + seg is unique per (CTA, segment) pair and < nslots,
 //  - the CTA interval [cta_of(first), cta_of(last)] of each segment is exactly the set of CTAs
-//    that flush a partial for it.
+//    that flush a partial for it,
+//  - with one block per head, the CTAs sharing a head's combine [ga, gb] form a non-empty
+//    sub-interval of the CTAs covering it, so their flags (index g + h) are unique slots.
 #include <cstdio>
 #include <cstdlib>
 #include <set>
@@ -45,6 +47,21 @@ static int check(int B, int H, int N, int L, int sms) {
     for (int cta = 0; cta < g.G; ++cta) {
       bool in = cta >= g0 && cta <= g1;
       if (in != (flushes.count({s, cta}) > 0)) { printf("scan interval mismatch seg %d cta %d\n", s, cta); return 1; }
+    }
+    if (g.nblk == 1) {
+      CombineRange cr = combine_range(s, g);
+      if (cr.g0 != g0 || cr.g1 != g1 || cr.ga < g0 || cr.gb > g1 || cr.ga > cr.gb) {
+        printf("combine range seg %d: [%d, %d] of [%d, %d]\n", s, cr.ga, cr.gb, g0, g1);
+        return 1;
+      }
+      // a CTA whose range starts inside the head is always among those sharing its combine
+      for (int cta = g0; cta <= g1; ++cta) {
+        long long tb = tile_begin(cta, g);
+        if (tb >= f && tb < f + seg_ntiles(s, g) && (cta < cr.ga || cta > cr.gb)) {
+          printf("combine range seg %d misses cta %d\n", s, cta);
+          return 1;
+        }
+      }
     }
   }
   return 0;
