@@ -406,6 +406,32 @@ def run_extra(args, name):
             evs[i + 1].record(stream)
         torch.cuda.synchronize()
         per += [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
+    # the same sequence of calls captured once in a CUDA graph and replayed: per-call device time
+    # without the host's per-call launch work (how a generation loop would issue the calls)
+    graph_ms = None
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(reps):
+                q, k, v = sets[i]
+                if kind == "stream":
+                    sv.sv_cache_step(q, k, v, S, z, commit=True, o=outs[i], ws=ws, stream=side)
+                else:
+                    sv.sv_linattn_fwd(q, k, v, o=outs[i], ws=ws, stream=side)
+        graph.replay()
+        side.synchronize()
+        nrep = max(1, args.steps // reps)
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga.record(side)
+        for _ in range(nrep):
+            graph.replay()
+        gb.record(side)
+        side.synchronize()
+        graph_ms = ga.elapsed_time(gb) / (nrep * reps)
+    del graph
+    torch.cuda.synchronize()
     if ws.status() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     per_ms = np.array(per)
@@ -416,6 +442,9 @@ def run_extra(args, name):
             "config": {"workload": desc}, "calls_timed": len(per), "ms_per_call_mean": ms,
             "ms_per_call_median": float(np.median(per_ms)), "ms_per_call_p90": float(np.percentile(per_ms, 90)),
             "hbm_gbs_alg": step_bytes / (ms / 1e3) / 1e9, "hbm_frac": step_bytes / (ms / 1e3) / 1e9 / hbm_gbs,
+            "graph": {"ms_per_call": graph_ms, "value": tokheads / (graph_ms / 1e3),
+                      "hbm_frac": step_bytes / (graph_ms / 1e3) / 1e9 / hbm_gbs,
+                      "timing": "the same calls captured in one CUDA graph, replayed; CUDA events"},
             "dtype": "bf16", "data": "synthetic (torch CUDA generator, seed 0)", "impl": "ours"}
     print(json.dumps(line), flush=True)
     return 0
@@ -424,7 +453,7 @@ def run_extra(args, name):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)

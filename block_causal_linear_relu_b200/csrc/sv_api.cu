@@ -231,11 +231,17 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
     SV_TRY(make_block_maps(mv, v, g, sv::kTile));
     SV_TRY(make_block_maps(mq, q, g, sv::kTile));
     SV_TRY(make_block_maps(mo, o, g, 32));
-    if (g.nblk == 1) {  // one block: a single fused launch
+    if (g.nblk == 1) {  // one block: a single launch, one cluster per head when the heads are few
       prof_mark(0, stream);
-      e = sv::launch_fused_bf16(mk, mv, mq, mo, g, partials, segcta, flags, pre, S_in, z_in, S_out, z_out, eps,
-                                status, stream);
-      if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
+      const int C = sv::cluster_size(g, di.sm_count);
+      if (C > 0) {
+        e = sv::launch_cluster_bf16(mk, mv, mq, mo, g, C, S_in, z_in, S_out, z_out, eps, status, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cluster kernel launch");
+      } else {
+        e = sv::launch_fused_bf16(mk, mv, mq, mo, g, partials, segcta, flags, pre, S_in, z_in, S_out, z_out, eps,
+                                  status, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
+      }
       prof_mark(1, stream);
       prof_mark(2, stream);
       prof_mark(3, stream);

@@ -27,6 +27,12 @@ cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const Bloc
                               const Geom& g, float* partials, int2* segcta, uint64_t* flags, void* ptiles,
                               const float* S_in, const float* z_in, float* S_out, float* z_out, float eps,
                               uint32_t* status, cudaStream_t st);
+// bf16, whole sequence in one block, few heads: one thread-block cluster of C CTAs per head.
+// cluster_size returns the C to use for this geometry (0: use launch_fused_bf16 instead).
+int cluster_size(const Geom& g, int sm_count);
+cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
+                                const Geom& g, int C, const float* S_in, const float* z_in, float* S_out,
+                                float* z_out, float eps, uint32_t* status, cudaStream_t st);
 // fp32 path
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
                              uint32_t* status, cudaStream_t st);

@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 
 #include <cstdlib>
+#include <mutex>
 #include <utility>
 
 #include "sv_internal.h"
@@ -476,10 +477,17 @@ __device__ __forceinline__ bool relu_q(uint8_t* smem, const Bars& b, long long k
   return true;
 }
 
+// Output staging: nbuf (1 or 2) sets of 4 warps x two 4 KB atoms starting at `base`.
+struct Staging {
+  uint8_t* base;
+  int nbuf;
+};
+
 // Epilogue of tile k for one warp: TMEM lanes 32q..32q+31 (q = warp % 4, tokens of the tile) and
 // output columns 64h..64h+63; numerator times 1 / (denominator + eps), bf16, into this warp's
-// swizzled 4 KB staging atom, then a TMA store clipped to the block.
-__device__ __forceinline__ bool epilogue_tile(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo,
+// swizzled 4 KB staging atom (alternating between buffers when there are two), then a TMA store
+// clipped to the block.
+__device__ __forceinline__ bool epilogue_tile(const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo,
                                               long long t, long long k, uint32_t tmem, int q, int h, int lane,
                                               float eps, uint32_t* status) {
   const TileCoord c = tile_coord(t, geo);
@@ -498,8 +506,13 @@ __device__ __forceinline__ bool epilogue_tile(uint8_t* smem, const Bars& b, cons
   __syncwarp();
   if (lane == 0) mbar_arrive(&b.acce[a]);  // the values are in registers: the accumulator is free
   const float inv = __frcp_rn(__uint_as_float(dr) + eps);
-  uint8_t* ob = smem + kOOff + q * kOWarpBytes + h * kAtomBytesO;
-  if (lane == 0) bulk_wait_read_all();  // this warp's previous store has finished reading the atom
+  uint8_t* ob = sg.base + ((sg.nbuf > 1 ? static_cast<int>(k & 1) * 4 : 0) + q) * kOWarpBytes + h * kAtomBytesO;
+  if (lane == 0) {  // the store that last read this atom (one or two tiles ago) has finished reading it
+    if (sg.nbuf > 1)
+      bulk_wait_read_all_but_one();
+    else
+      bulk_wait_read_all();
+  }
   __syncwarp();
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
@@ -522,34 +535,35 @@ __device__ __forceinline__ bool epilogue_tile(uint8_t* smem, const Bars& b, cons
     if (row0 < blen) {
       const bool lst = use_last_map(c, geo);
       tma_store_4d(lst ? m.b_last : m.b_main, ob, h * 64, row0, lst ? 0 : c.blk, c.bh);
-      bulk_commit();
     }
+    bulk_commit();  // one group per tile (possibly empty), so "all but the latest" means the previous tile
   }
   return true;
 }
 
 // Warps 0-3: epilogue of output columns 0..63 of every tile.
-__device__ void epilogue_role(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
+__device__ void epilogue_role(const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
                               long long te, uint32_t tmem, int warp, int lane, float eps, uint32_t* status) {
   long long k = 0;
   for (long long t = tb; t < te; ++t, ++k)
-    if (!epilogue_tile(smem, b, m, geo, t, k, tmem, warp & 3, 0, lane, eps, status)) break;
+    if (!epilogue_tile(sg, b, m, geo, t, k, tmem, warp & 3, 0, lane, eps, status)) break;
   if (lane == 0) bulk_wait_all();
 }
 
-// Warps 4-7: ReLU of the Q tiles, running up to kStages tiles ahead, and (D > 64) the epilogue of
-// output columns 64..127. Tile k + kStages is ReLU'd after the epilogue of tile k: its stage was
-// freed by the MMAs of tile k, which the epilogue has waited for, so the order cannot deadlock.
-__device__ void relu_epi_role(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
-                              long long te, bool two_atoms, uint32_t tmem, int warp, int lane, float eps,
-                              uint32_t* status) {
+// Warps 4-7: ReLU of the Q tiles, running up to kStages tiles ahead (relu_done <= kStages of them
+// already done), and (D > 64) the epilogue of output columns 64..127. Tile k + kStages is ReLU'd
+// after the epilogue of tile k: its stage was freed by the MMAs of tile k, which the epilogue has
+// waited for, so the order cannot deadlock.
+__device__ void relu_epi_role(uint8_t* smem, const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo,
+                              long long tb, long long te, int relu_done, bool two_atoms, uint32_t tmem, int warp,
+                              int lane, float eps, uint32_t* status) {
   const int r = static_cast<int>(threadIdx.x) - 128;
   const long long n = te - tb;
-  long long kr = 0;
+  long long kr = relu_done;  // tiles [0, relu_done) were ReLU'd by the caller
   bool ok = true;
   for (; kr < n && kr < kStages && ok; ++kr) ok = relu_q(smem, b, kr, two_atoms, r, lane, status);
   for (long long k = 0; k < n && ok; ++k) {
-    if (two_atoms) ok = epilogue_tile(smem, b, m, geo, tb + k, k, tmem, warp & 3, 1, lane, eps, status);
+    if (two_atoms) ok = epilogue_tile(sg, b, m, geo, tb + k, k, tmem, warp & 3, 1, lane, eps, status);
     if (ok && kr < n) ok = relu_q(smem, b, kr++, two_atoms, r, lane, status);
   }
   if (two_atoms && lane == 0) bulk_wait_all();
@@ -655,11 +669,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       ot::produce(smem, b, m, geo, tb, te, pre, two_atoms, ptiles, nullptr, 0, status);
     }
   } else if (warp >= 4 && warp < 8) {
-    ot::relu_epi_role(smem, b, m, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
+    ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, m, geo, tb, te, 0, two_atoms, tmem, warp, lane,
+                      eps, status);
   } else if (warp == kWarpMma) {
     if (lane == 0) ot::mma_role(smem, b, geo, tb, te, two_atoms, tmem, status);
   } else {
-    ot::epilogue_role(smem, b, m, geo, tb, te, tmem, warp, lane, eps, status);
+    ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, b, m, geo, tb, te, tmem, warp, lane, eps, status);
   }
   persistent_teardown(tmem, warp);
 }
@@ -856,6 +871,55 @@ __device__ void combine_load_cache(const Geom& geo, const float* S_in, const flo
     for (int d = tid; d < D; d += nthr) sZ[d] = __ldcg(z_in + static_cast<size_t>(bh) * D + d);
 }
 
+// The same two steps for a share whose bounds are multiples of 4 (float4 along e when the cache is
+// 16-byte aligned; the API only promises 4-byte alignment, so otherwise element by element).
+__device__ void combine_load_cache_q(const Geom& geo, const float* S_in, const float* z_in, int bh, int r0, int r1,
+                                     float* sS, float* sZ, int tid, int nthr) {
+  const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1), nq = ns / 4;
+  if (S_in != nullptr) {
+    const float* src = S_in + static_cast<size_t>(bh) * D * D + r0;
+    if ((reinterpret_cast<uintptr_t>(S_in) & 15u) == 0u) {
+      for (int i = tid; i < D * nq; i += nthr) {
+        const int d = i / nq, j = (i - d * nq) * 4;
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(d) * D + j));
+        sS[(j + 0) * ld + d] = v.x;
+        sS[(j + 1) * ld + d] = v.y;
+        sS[(j + 2) * ld + d] = v.z;
+        sS[(j + 3) * ld + d] = v.w;
+      }
+    } else {
+      for (int i = tid; i < D * ns; i += nthr) {
+        const int d = i / ns, j = i - d * ns;
+        sS[j * ld + d] = __ldcg(src + static_cast<size_t>(d) * D + j);
+      }
+    }
+  }
+  if (z_in != nullptr && r0 <= kZRow && kZRow < r1)
+    for (int d = tid; d < D; d += nthr) sZ[d] = __ldcg(z_in + static_cast<size_t>(bh) * D + d);
+}
+
+__device__ void combine_store_cache_q(const Geom& geo, float* S_out, float* z_out, int bh, int r0, int r1,
+                                      const float* sS, const float* sZ, int tid, int nthr) {
+  const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1), nq = ns / 4;
+  if (S_out != nullptr) {
+    float* dst = S_out + static_cast<size_t>(bh) * D * D + r0;
+    if ((reinterpret_cast<uintptr_t>(S_out) & 15u) == 0u) {
+      for (int i = tid; i < D * nq; i += nthr) {
+        const int d = i / nq, j = (i - d * nq) * 4;
+        *reinterpret_cast<float4*>(dst + static_cast<size_t>(d) * D + j) =
+            make_float4(sS[(j + 0) * ld + d], sS[(j + 1) * ld + d], sS[(j + 2) * ld + d], sS[(j + 3) * ld + d]);
+      }
+    } else {
+      for (int i = tid; i < D * ns; i += nthr) {
+        const int d = i / ns, j = i - d * ns;
+        dst[static_cast<size_t>(d) * D + j] = sS[j * ld + d];
+      }
+    }
+  }
+  if (z_out != nullptr && r0 <= kZRow && kZRow < r1)
+    for (int d = tid; d < D; d += nthr) z_out[static_cast<size_t>(bh) * D + d] = sZ[d];
+}
+
 // Step 2 (once the head's partial slots exist): each row = cache + the slots of CTAs g0..g1 in
 // ascending order, written as the bf16 B operand of the output GEMM; the sums replace the cache
 // values in sS / sZ for step 3. Each thread takes two (row, quad) items per pass and keeps up to 8
@@ -935,16 +999,16 @@ __device__ void combine_sum(const Geom& geo, const float* __restrict__ partials,
 // Step 3 (after the prefix rows are published; nothing in this launch reads the outgoing cache):
 // the share's rows of the outgoing cache from sS / sZ.
 __device__ void combine_store_cache(const Geom& geo, float* S_out, float* z_out, int bh, int r0, int r1,
-                                    const float* sS, const float* sZ) {
+                                    const float* sS, const float* sZ, int tid, int nthr) {
   const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1);
   if (S_out != nullptr) {
-    for (int i = threadIdx.x; i < D * ns; i += kThreads) {
+    for (int i = tid; i < D * ns; i += nthr) {
       const int d = i / ns, j = i - d * ns;
       S_out[(static_cast<size_t>(bh) * D + d) * D + r0 + j] = sS[j * ld + d];
     }
   }
   if (z_out != nullptr && r0 <= kZRow && kZRow < r1)
-    for (int d = threadIdx.x; d < D; d += kThreads) z_out[static_cast<size_t>(bh) * D + d] = sZ[d];
+    for (int d = tid; d < D; d += nthr) z_out[static_cast<size_t>(bh) * D + d] = sZ[d];
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1047,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       st_release_u64(combined + g + h, tag);
     }
-    if (s_ok) combine_store_cache(geo, S_out, z_out, h, r0, r1, sS, sZ);
+    if (s_ok) combine_store_cache(geo, S_out, z_out, h, r0, r1, sS, sZ, threadIdx.x, kThreads);
     __syncthreads();
   }
   fence_proxy_async_smem();  // the combine scratch is next written by TMA copies (async proxy)
@@ -1059,15 +1123,238 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpProducer) {
       if (lane == 0) ot::produce(smem, ob, mqo, geo, tb, te, pre, two_atoms, ptiles, combined, tag, status);
     } else if (warp >= 4 && warp < 8) {
-      ot::relu_epi_role(smem, ob, mqo, geo, tb, te, two_atoms, tmem, warp, lane, eps, status);
+      ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, ob, mqo, geo, tb, te, 0, two_atoms, tmem, warp, lane,
+                        eps, status);
     } else if (warp == kWarpMma) {
       if (lane == 0) ot::mma_role(smem, ob, geo, tb, te, two_atoms, tmem, status);
     } else {
-      ot::epilogue_role(smem, ob, mqo, geo, tb, te, tmem, warp, lane, eps, status);
+      ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, ob, mqo, geo, tb, te, tmem, warp, lane, eps, status);
     }
   } else if (warp == kWarpProducer && lane == 0) {
     for (int i = 0; i < pre; ++i) mbar_wait(&ob.qfull[i], 0, status, 0x2180u);  // prefilled loads land
   }
+  persistent_teardown(tmem, warp);
+}
+
+// ------------------------------------------------------------------------------------------
+// 5. one block per head with one thread-block cluster per head (few heads, e.g. a streaming step)
+// ------------------------------------------------------------------------------------------
+// Cluster h (C CTAs) owns head h; rank r reduces tiles [r*tph/C, (r+1)*tph/C) of the head into
+// TMEM exactly as the state roles do, then drains its partial state into its own shared memory.
+// After a cluster barrier each rank sums its share of prefix rows over the C partials, read in rank
+// order through distributed shared memory, adds the incoming cache, and writes the bf16 rows into
+// the prefix tile of every rank of the cluster. After a second cluster barrier every rank holds
+// the whole prefix tile and runs the output roles on its tiles; the outgoing cache is written from
+// the fp32 sums. No global round trip and no flag sits between the reduction and the output.
+// Every thread reaches both cluster barriers on every path (the roles only leave their loops on
+// a failed bounded wait), and no shared memory of another rank is touched after the second one.
+namespace cl {
+constexpr int kMinCluster = 4;
+constexpr int kMaxCluster = 8;
+constexpr int kPartOff = ot::kBOff + kPTileBytes;                // partial [129][128] fp32 (row e, column d)
+constexpr int kPartBytes = kPartRows * kDPad * 4;
+static_assert(kPartOff + kPartBytes <= fu::kRegion, "partial state overflows the stage region");
+static_assert(kPartOff >= ot::kBOff + kPTileBytes && kPartOff % 1024 == 0, "partial overlaps the prefix tile");
+static_assert(kPartOff + 2 * 4 * ot::kOWarpBytes <= fu::kRegion, "double-buffered output staging overflows");
+constexpr int kShareRowsMax = (kPTileRows + kMinCluster - 1) / kMinCluster;
+constexpr int kScratchOff = fu::kRegion;                          // incoming-cache share, transposed
+constexpr int kScratchZOff = kScratchOff + kShareRowsMax * (kDPad + 1) * 4;
+constexpr int kBarOff = (kScratchZOff + kDPad * 4 + 7) / 8 * 8;
+constexpr int kSmem = kBarOff + 512 + 1024;
+static_assert(kSmem <= 227 * 1024, "cluster kernel shared memory");
+}  // namespace cl
+
+// Epilogue warps 0-3: the single accumulator of this rank (TMEM lanes = key feature d) into the
+// partial [e][d] in shared memory; row kZRow holds z.
+__device__ void cl_drain_partial(const st::Bars& b, uint32_t tmem, int warp, int lane, float* part,
+                                 uint32_t* status) {
+  const int d = warp * 32 + lane;
+  const bool ok = mbar_wait(&b.accf[0], 0, status, 0x3400u);
+  if (!warp_all(ok)) return;
+  tc_fence_after();
+  const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t rr[2][32];
+    uint32_t zr = 0;
+    tmem_ld_x32(ta + h * 64, rr[0]);
+    tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+    if (h == 1) tmem_ld_x1(ta + 128, zr);
+    tmem_wait_ld();
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) part[(h * 64 + cc * 32 + jj) * kDPad + d] = __uint_as_float(rr[cc][jj]);
+    if (h == 1) part[kZRow * kDPad + d] = __uint_as_float(zr);
+  }
+  tc_fence_before();
+}
+
+// This rank's share of the head's prefix rows: sum of the C partials (rank order) + cache, bf16 rows
+// written into every rank's prefix tile; the fp32 sums stay in sS / sZ for the outgoing cache.
+__device__ void cl_combine(const Geom& geo, uint32_t part_s, uint32_t ptile_s, int C, int me, bool has_S,
+                           bool has_z, int r0, int r1, float* sS, float* sZ, int tid, int nthr) {
+  const int D = geo.D, ld = D + 1;
+  // two (row, quad) items per thread and pass, the C partial values of both in flight at once
+  for (int base = r0 * 32 + tid; base < r1 * 32; base += 2 * nthr) {
+    float4 p[2][cl::kMaxCluster];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int it = base + x * nthr;
+      const int e = it >> 5, d0 = (it & 31) * 4;
+      const uint32_t off = static_cast<uint32_t>((e * kDPad + d0) * 4);
+#pragma unroll
+      for (int q = 0; q < cl::kMaxCluster; ++q)
+        if (q < C && it < r1 * 32 && e < kPartRows)
+          p[x][q] = q == me ? ld_shared_f4(part_s + off)
+                            : ld_shared_cluster_f4(mapa_shared(part_s + off, static_cast<uint32_t>(q)));
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int it = base + x * nthr;
+      if (it >= r1 * 32) break;
+      const int e = it >> 5, d0 = (it & 31) * 4;
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+      if (e < kPartRows) {
+#pragma unroll
+        for (int q = 0; q < cl::kMaxCluster; ++q) {
+          if (q < C) {
+            a[0] += p[x][q].x;
+            a[1] += p[x][q].y;
+            a[2] += p[x][q].z;
+            a[3] += p[x][q].w;
+          }
+        }
+        if (e < D) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (d0 + u < D) {
+              float* c = &sS[(e - r0) * ld + d0 + u];
+              if (has_S) a[u] += *c;
+              *c = a[u];
+            }
+          }
+        } else if (e == kZRow) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (d0 + u < D) {
+              if (has_z) a[u] += sZ[d0 + u];
+              sZ[d0 + u] = a[u];
+            }
+          }
+        }
+      }
+      uint2 w;
+      w.x = pack_bf16x2(a[0], a[1]);
+      w.y = pack_bf16x2(a[2], a[3]);
+      const uint32_t off = static_cast<uint32_t>((d0 >> 6) * (kPTileRows * 128) + e * 128 +
+                                                 ((((d0 & 63) >> 3) ^ (e & 7)) << 4) + (d0 & 7) * 2);
+      for (int q = 0; q < C; ++q) {
+        if (q == me)
+          st_shared_u2(ptile_s + off, w);
+        else
+          st_shared_cluster_u2(mapa_shared(ptile_s + off, static_cast<uint32_t>(q)), w);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    cluster_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
+                        const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
+                        const __grid_constant__ CUtensorMap q_main, const __grid_constant__ CUtensorMap q_last,
+                        const __grid_constant__ CUtensorMap o_main, const __grid_constant__ CUtensorMap o_last,
+                        const Geom geo, const float* S_in, const float* z_in, float* S_out, float* z_out,
+                        const float eps, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + cl::kBarOff);
+  const st::Bars sb = st::bars_at(barmem);
+  const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + st::kNumBars + ot::kNumBars);
+  float* part = reinterpret_cast<float*>(smem + cl::kPartOff);
+  float* sS = reinterpret_cast<float*>(smem + cl::kScratchOff);
+  float* sZ = reinterpret_cast<float*>(smem + cl::kScratchZOff);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int C = static_cast<int>(gridDim.x) / geo.BH;  // cluster size (grid = B*H clusters of C CTAs)
+  const int bh = static_cast<int>(cluster_id_x());
+  const int r = static_cast<int>(cluster_ctarank());
+  const long long tb = static_cast<long long>(bh) * geo.tph + static_cast<long long>(r) * geo.tph / C;
+  const long long te = static_cast<long long>(bh) * geo.tph + static_cast<long long>(r + 1) * geo.tph / C;
+  const int r0 = 4 * (r * (kPTileRows / 4) / C), r1 = 4 * ((r + 1) * (kPTileRows / 4) / C);  // whole quads
+  const bool two_atoms = geo.D > 64;
+  const Maps4 mkv{&k_main, &k_last, &v_main, &v_last};
+  const Maps4 mqo{&q_main, &q_last, &o_main, &o_last};
+  if (threadIdx.x == 0) {
+    st::init_bars(sb);
+    ot::init_bars(ob, two_atoms);
+    fence_mbar_init();
+  }
+  st::init_smem(smem, two_atoms, kThreads);
+  if (warp == kWarpProducer && lane == 0) {
+    prefetch_maps(mkv);
+    prefetch_maps(mqo);
+  }
+  const uint32_t tmem = persistent_setup(tmem_slot, warp);
+  griddep_wait();  // the previous kernel in the stream may still write q, k, v or the cache
+  if (threadIdx.x == 0) griddep_launch_dependents();
+
+  // phase 1: this rank's partial state; the epilogue warps first fetch the cache share
+  if (warp == kWarpProducer) {
+    if (lane == 0) st::produce(smem, sb, mkv, geo, tb, te, two_atoms, false, status);
+  } else if (warp >= 4 && warp < 8) {
+    st::relu_role(smem, sb, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) st::mma_role(smem, sb, geo, tb, te, tmem, status);
+  } else {
+    combine_load_cache_q(geo, S_in, z_in, bh, r0, r1, sS, sZ, threadIdx.x, 128);
+    cl_drain_partial(sb, tmem, warp, lane, part, status);
+  }
+  __syncthreads();
+
+  // phase 2: Q stages fill while the cluster exchanges the partial states. The Q loads are issued
+  // after the first cluster barrier: issued before it, they delayed its release by about 1 us.
+  const int pre = static_cast<int>(te - tb < ot::kStages ? te - tb : ot::kStages);  // Q tiles prefilled
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (warp == kWarpProducer && lane == 0) ot::prefill(smem, ob, mqo, geo, tb, te, two_atoms);
+  // The ReLU warps rewrite the prefilled Q tiles that have already landed while the other warps
+  // combine (the combine is bound by distributed-shared-memory bandwidth, not by its thread count);
+  // tiles still in flight are left to phase 3 so that the second barrier never waits for Q.
+  int relu_done = 0;
+  if (warp >= 4 && warp < 8) {
+    while (relu_done < pre && warp_all(mbar_try_wait(&ob.qfull[relu_done], 0)) &&
+           ot::relu_q(smem, ob, relu_done, two_atoms, threadIdx.x - 128, lane, status))
+      ++relu_done;
+  } else {
+    const int tid = warp < 4 ? static_cast<int>(threadIdx.x) : 128 + (warp - kWarpProducer) * 32 + lane;
+    cl_combine(geo, smem_u32(part), smem_u32(smem + ot::kBOff), C, r, S_in != nullptr, z_in != nullptr, r0, r1, sS,
+               sZ, tid, 192);
+  }
+  fence_proxy_async_all();
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  fence_proxy_async_all();  // the prefix tile written by the cluster -> tcgen05.mma reads (async proxy)
+  tc_fence_after();
+
+  // phase 3: output of this rank's tiles against the resident prefix tile. The partial states are
+  // no longer read by any rank, so their memory becomes double-buffered output staging. (After a
+  // failed wait anywhere in the grid every later wait returns at once, so phase 3 runs regardless.)
+  const ot::Staging sg{smem + cl::kPartOff, 2};
+  if (warp == kWarpProducer) {
+    if (lane == 0) ot::produce(smem, ob, mqo, geo, tb, te, pre, two_atoms, nullptr, nullptr, 0, status);
+  } else if (warp >= 4 && warp < 8) {
+    ot::relu_epi_role(smem, sg, ob, mqo, geo, tb, te, relu_done, two_atoms, tmem, warp, lane, eps, status);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) ot::mma_role(smem, ob, geo, tb, te, two_atoms, tmem, status);
+  } else {
+    ot::epilogue_role(sg, ob, mqo, geo, tb, te, tmem, warp, lane, eps, status);
+  }
+  // the outgoing cache last: nothing in this launch reads it, and its stores drain with the output
+  // (lanes 1..31 of the producer and MMA warps wait for lane 0 first, so they do not compete with it)
+  __syncwarp();
+  combine_store_cache_q(geo, S_out, z_out, bh, r0, r1, sS, sZ, threadIdx.x, kThreads);
   persistent_teardown(tmem, warp);
 }
 
@@ -1217,6 +1504,8 @@ cudaError_t set_kernel_attributes() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fu::kSmem);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(cluster_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cl::kSmem);
+  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(out_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(state_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateF32Smem);
@@ -1271,6 +1560,67 @@ cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const Bloc
   return cudaLaunchKernelEx(&cfg, fused_bf16_kernel, k.main, k.last, v.main, v.last, q.main, q.last, o.main, o.last,
                             g, partials, segcta, flags, flags + g.nslots, static_cast<uint8_t*>(ptiles), S_in, z_in,
                             S_out, z_out, eps, status);
+}
+
+// Cluster size for the cluster kernel, or 0 when the flag-synchronised kernel should run: the
+// largest C in [4, 8] such that every rank gets a tile, B*H clusters of C CTAs can all be resident
+// (as the occupancy query reports for this device), and they occupy at least 3/4 of the SMs.
+int cluster_size(const Geom& g, int sm_count) {
+  static std::mutex mu;
+  static int max_active[64][cl::kMaxCluster + 1];
+  static bool known[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!known[dev]) {
+    for (int c = cl::kMinCluster; c <= cl::kMaxCluster; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(c * 16);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = cl::kSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = c;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, cluster_bf16_kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+      max_active[dev][c] = n;
+    }
+    known[dev] = true;
+  }
+  for (int c = cl::kMaxCluster; c >= cl::kMinCluster; --c) {
+    if (c > g.tph || max_active[dev][c] < g.BH) continue;
+    if (static_cast<long long>(g.BH) * c * 4 < static_cast<long long>(sm_count) * 3) continue;
+    return c;
+  }
+  return 0;
+}
+
+cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
+                                const Geom& g, int C, const float* S_in, const float* z_in, float* S_out,
+                                float* z_out, float eps, uint32_t* status, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(g.BH * C));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = cl::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, cluster_bf16_kernel, k.main, k.last, v.main, v.last, q.main, q.last, o.main,
+                            o.last, g, S_in, z_in, S_out, z_out, eps, status);
 }
 
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,

@@ -62,7 +62,8 @@ extern "C" sv_status sv_cache_step_noalloc(const void* q, const void* k, const v
       void* p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess || p == nullptr)
-        return sv::set_last_error(SV_ERR_CUDA, "sv_cache_step_noalloc: cudaGetSymbolAddress of the static scratch failed");
+        return sv::set_last_error(SV_ERR_CUDA,
+                                  "sv_cache_step_noalloc: cudaGetSymbolAddress of the static scratch failed");
       g_scratch_addr[dev] = p;
     }
     ws = g_scratch_addr[dev];

@@ -31,8 +31,8 @@ __global__ void __launch_bounds__(128, 1) selftest_wait_kernel(uint32_t* status)
 extern "C" sv_status sv_selftest_wait_timeout(void* ws, size_t ws_bytes, sv_stream_t stream) {
   if (ws == nullptr || ws_bytes < static_cast<size_t>(sv::kHeaderBytes) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u) != 0u)
-    return sv::set_last_error(SV_ERR_INVALID_ARG,
-                              "sv_selftest_wait_timeout: ws must be a 256-byte aligned workspace of at least 256 bytes");
+    return sv::set_last_error(
+        SV_ERR_INVALID_ARG, "sv_selftest_wait_timeout: ws must be a 256-byte aligned workspace of at least 256 bytes");
   selftest_wait_kernel<<<1, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(ws));
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return sv::set_last_error(SV_ERR_CUDA, cudaGetErrorString(e));

@@ -115,6 +115,26 @@ def test_bf16_many_tiles_per_cta(sv):
     assert oracle.max_rel_err(host(z_out), z_ref) < TOL_CACHE
 
 
+# --------------------------------------------------------------------------------------------
+# one block per head with 14..26 heads: one thread-block cluster of 4..8 CTAs per head exchanges
+# the partial states through distributed shared memory; incoming cache, in-place update
+# --------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("B,H,N,D", [(1, 20, 800, 128), (2, 10, 2760, 128), (1, 24, 1000, 112),
+                                     (1, 20, 1500, 64), (1, 20, 700, 96)])
+def test_one_block_few_heads_with_cache(sv, B, H, N, D):
+    st, (q, k, v) = inputs((B, H, N, D), 5, "bf16")
+    g = np.random.default_rng(7)
+    S0 = g.standard_normal((B, H, D, D)).astype(np.float32) * 10
+    z0 = np.abs(g.standard_normal((B, H, D))).astype(np.float32) * 100
+    S = torch.from_numpy(S0).cuda()
+    z = torch.from_numpy(z0).cuda()
+    o = run_bc(sv, st, "bf16", N, S_in=S, z_in=z, S_out=S, z_out=z)
+    ref, S_ref, z_ref = oracle.block_causal_attn(q, k, v, N, EPS, S0.astype(np.float64), z0.astype(np.float64))
+    assert oracle.max_rel_err(host(o), ref) < TOL["bf16"]
+    assert oracle.max_rel_err(host(S), S_ref) < TOL_CACHE
+    assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
+
+
 def test_bf16_error_is_well_inside_tolerance(sv):
     # the bf16 path's only rounding steps are the bf16 prefix operand and the bf16 output:
     # the measured error should sit near 1e-3, an order below the 2e-2 bar
