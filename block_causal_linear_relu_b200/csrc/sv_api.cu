@@ -251,7 +251,7 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
     e = sv::launch_state_bf16(mk, mv, g, partials, segcta, status, stream);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
     prof_mark(1, stream);
-    e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, pre, nullptr, stream);
+    e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, pre, nullptr, status + 6, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     prof_mark(2, stream);
     e = sv::launch_out_bf16(mq, mo, g, pre, eps, status, stream);
@@ -264,7 +264,7 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
                              status, stream);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
     prof_mark(1, stream);
-    e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, nullptr, p32, stream);
+    e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, nullptr, p32, status + 6, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     prof_mark(2, stream);
     e = sv::launch_out_f32(static_cast<const float*>(q), static_cast<float*>(o), g, p32, eps, status, stream);
@@ -376,7 +376,7 @@ sv_status sv_block_state_update(const void* k, const void* v, int B, int H, int 
                              status, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
-  e = sv::launch_scan(partials, segcta, g, S, z, S, z, nullptr, nullptr, s);
+  e = sv::launch_scan(partials, segcta, g, S, z, S, z, nullptr, nullptr, status + 6, s);
   if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
   return SV_OK;
 }

@@ -29,6 +29,7 @@ constexpr int kPartRows = 129;          // S^T rows (value feature e) + the z ro
 constexpr int kPTileRows = 144;         // B operand rows of the output GEMM: 128 + z row + 15 zero rows
 constexpr int kPTileBytes = kPTileRows * kDPad * 2;          // one bf16 prefix tile, 36,864 B
 constexpr int kPartBytes = kPartRows * kDPad * 4;            // one fp32 partial, 66,048 B
+constexpr int kOutChunk = 4;      // tiles per dynamically handed-out output chunk
 constexpr int kHeaderBytes = 256;                            // status word(s) at the workspace start
 
 constexpr uint32_t kDevTimeout = 0x80000000u;                // status bit: a bounded wait expired
@@ -48,6 +49,7 @@ struct Geom {
   long long T;  // total tiles
   int nseg;     // BH * nblk
   int nslots;   // G + nseg - 1
+  long long tdyn;  // output pass: the last tdyn tiles are handed out dynamically (multiple of kOutChunk)
 };
 
 SV_HD int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
@@ -134,7 +136,14 @@ inline bool make_geom(Geom& q, int B, int H, int N, int D, int block_len, int sm
   if (nseg > (1ll << 30)) return false;
   q.nseg = static_cast<int>(nseg);
   q.nslots = q.G + q.nseg - 1;
+  // The output pass splits [0, T - tdyn) statically over the G CTAs and hands out the remaining
+  // tdyn tiles in chunks of kOutChunk to whichever CTA finishes first (about 1/8 of the tiles,
+  // once every CTA has at least 8 static tiles).
+  q.tdyn = q.T >= 9ll * q.G ? (q.T / 8) / kOutChunk * kOutChunk : 0;
   return true;
 }
+
+// Static output range of CTA g: [out_tile_begin(g), out_tile_begin(g + 1)) of [0, T - tdyn).
+SV_HD long long out_tile_begin(int g, const Geom& q) { return static_cast<long long>(g) * (q.T - q.tdyn) / q.G; }
 
 }  // namespace sv

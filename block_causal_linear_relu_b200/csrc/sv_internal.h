@@ -39,8 +39,10 @@ cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, floa
 cudaError_t launch_out_f32(const float* q, float* o, const Geom& g, const float* p32, float eps,
                            uint32_t* status, cudaStream_t st);
 // both paths: combine partials, inclusive prefix over blocks, optional final cache
+// out_chunks: the output kernel's dynamic-chunk counter (workspace header bytes 24..27), reset here.
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
-                        float* S_out, float* z_out, void* ptiles_bf16, float* p32, cudaStream_t st);
+                        float* S_out, float* z_out, void* ptiles_bf16, float* p32, uint32_t* out_chunks,
+                        cudaStream_t st);
 
 // Records `msg` as the calling thread's sv_last_error() text and returns `status`.
 sv_status set_last_error(sv_status status, const char* msg);

@@ -374,13 +374,29 @@ __device__ __forceinline__ void load_q(uint8_t* smem, const Bars& b, const Maps4
   if (two_atoms) tma_load_4d(stg + kAtomBytes, mq, &b.qfull[s], 64, c.tok0, cb, c.bh, pol);
 }
 
-// Q was final before the state reduction ran, so the first stages can fill before the prefix
-// exists. Returns how many tiles were issued.
-__device__ int prefill(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb, long long te,
-                       bool two_atoms) {
+// The output tiles of a CTA: its static range [tb, te), then, when `counter` is set, chunks of
+// kDynChunk tiles of [dyn_begin, dyn_end) claimed through an atomic counter by whichever CTA gets
+// there first (output tiles are independent, so the result does not depend on who computes what).
+// The producer walks the sequence and writes the k-th tile's index into ring[k % kRing] before
+// the barrier the other roles wait on for that tile (qfull); -1 ends the sequence.
+constexpr int kRing = 8;
+constexpr int kDynChunk = kOutChunk;
+struct Seq {
+  long long tb, te;
+  long long dyn_begin, dyn_end;
+  uint32_t* counter;
+  volatile long long* ring;
+};
+
+// Q was final before the state reduction ran, so the first stages of the static range can fill
+// before the prefix exists. Returns how many tiles were issued.
+__device__ int prefill(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, const Seq& sq, bool two_atoms) {
   const uint64_t pol = policy_evict_first();
-  const int pre = static_cast<int>(te - tb < kStages ? te - tb : kStages);
-  for (int i = 0; i < pre; ++i) load_q(smem, b, m, geo, tb + i, i, two_atoms, pol);
+  const int pre = static_cast<int>(sq.te - sq.tb < kStages ? sq.te - sq.tb : kStages);
+  for (int i = 0; i < pre; ++i) {
+    sq.ring[i] = sq.tb + i;
+    load_q(smem, b, m, geo, sq.tb + i, i, two_atoms, pol);
+  }
   return pre;
 }
 
@@ -390,13 +406,21 @@ __device__ int prefill(uint8_t* smem, const Bars& b, const Maps4& m, const Geom&
 // once every CTA sharing the head's combine has published its rows (value `tag`). With ptiles ==
 // nullptr the prefix tiles are already in shared memory (buffer j & 1 for the j-th segment) and
 // are only signalled to the MMA warp.
-__device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long tb, long long te,
-                        int pre, bool two_atoms, const uint8_t* __restrict__ ptiles, const uint64_t* combined,
-                        uint64_t tag, uint32_t* status) {
+__device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, const Seq& sq, int pre,
+                        bool two_atoms, const uint8_t* __restrict__ ptiles, const uint64_t* combined, uint64_t tag,
+                        uint32_t* status) {
   const uint64_t pol = policy_evict_first();
   int k = 0, j = 0, prev = -1;
   bool ok = true;
-  for (long long t = tb; t < te && ok; ++t, ++k) {
+  long long t = sq.tb, end = sq.te;
+  for (;; ++t, ++k) {
+    if (t >= end) {  // static range done: claim the next chunk of the dynamic range, if any
+      if (sq.counter == nullptr) break;
+      const long long c0 = sq.dyn_begin + static_cast<long long>(atomicAdd(sq.counter, 1u)) * kDynChunk;
+      if (c0 >= sq.dyn_end) break;
+      t = c0;
+      end = c0 + kDynChunk < sq.dyn_end ? c0 + kDynChunk : sq.dyn_end;
+    }
     const TileCoord c = tile_coord(t, geo);
     if (c.seg != prev && ptiles == nullptr) {  // the caller already placed the tile in buffer j & 1
       mbar_arrive(&b.bfull[j & 1]);
@@ -406,10 +430,10 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
       const int bb = j & 1;
       if (combined != nullptr) {
         const CombineRange cr = combine_range(c.seg, geo);
-        if (!wait_flags(combined, cr.ga + c.seg, cr.gb + c.seg, tag, status, 0x2200u)) break;
+        if (!wait_flags(combined, cr.ga + c.seg, cr.gb + c.seg, tag, status, 0x2200u)) { ok = false; break; }
         fence_proxy_async_global();  // prefix tile written by other CTAs -> bulk copy below
       }
-      if (!mbar_wait(&b.bempty[bb], ((j >> 1) & 1) ^ 1, status, 0x1100u | bb)) break;
+      if (!mbar_wait(&b.bempty[bb], ((j >> 1) & 1) ^ 1, status, 0x1100u | bb)) { ok = false; break; }
       mbar_expect_tx(&b.bfull[bb], kPTileBytes);
       bulk_load(smem + kBOff + bb * kPTileBytes, ptiles + static_cast<size_t>(c.seg) * kPTileBytes, kPTileBytes,
                 &b.bfull[bb]);
@@ -418,32 +442,53 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
     }
     if (k >= pre) {
       const int s = k % kStages;
-      if (!mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) break;
+      if (!mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) { ok = false; break; }
+      sq.ring[k % kRing] = t;
       load_q(smem, b, m, geo, t, s, two_atoms, pol);
     }
   }
-  for (int i = (k > kStages ? k - kStages : 0); i < (k > pre ? k : pre); ++i)
+  if (ok) {  // end of the sequence: a plain arrival completes the next stage's qfull with index -1
+    const int s = k % kStages;
+    if (k < pre || mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1140u | s)) {
+      sq.ring[k % kRing] = -1;
+      mbar_arrive(&b.qfull[s]);
+      ++k;
+    }
+  }
+  for (int i = (k > kStages ? k - kStages : 0); i < k; ++i)
     mbar_wait(&b.qfull[i % kStages], (i / kStages) & 1, status, 0x1180u);
   for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&b.bfull[i & 1], (i >> 1) & 1, status, 0x1190u);
 }
 
-__device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, bool two_atoms,
-                         uint32_t tmem, uint32_t* status) {
+__device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, const Seq& sq, bool two_atoms, uint32_t tmem,
+                         uint32_t* status) {
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, kPTileRows, false, false);
   const int ksteps = two_atoms ? 8 : 4;
-  int k = 0, j = 0, prev = -1, bb = 0;
-  for (long long t = tb; t < te; ++t, ++k) {
+  int j = 0, prev = -1, bb = 0;
+  for (int k = 0;; ++k) {
+    const int s = k % kStages;
+    const uint32_t ph = (k / kStages) & 1;
+    const int a = k & 1;
+    if (!mbar_wait(&b.qfull[s], ph, status, 0x1310u | s)) break;
+    const long long t = sq.ring[k % kRing];
+    if (t < 0) {
+      // End of the sequence, announced on this accumulator's barrier under the same flow control
+      // as a tile: first the epilogue must have released the accumulator's previous use (tile
+      // k - 2), or the barrier could run two phases ahead of a slow epilogue, which would then
+      // wait for a parity it already missed. The commit arrives once every MMA issued so far has
+      // retired.
+      if (!mbar_wait(&b.acce[a], ((k >> 1) & 1) ^ 1, status, 0x1340u | a)) break;
+      mma_commit(&b.accf[a]);
+      break;
+    }
     const TileCoord c = tile_coord(t, geo);
     if (c.seg != prev) {
+      if (j > 0) mma_commit(&b.bempty[(j - 1) & 1]);  // the previous prefix tile is free once its MMAs retire
       bb = j & 1;
       if (!mbar_wait(&b.bfull[bb], (j >> 1) & 1, status, 0x1300u | bb)) break;
       ++j;
       prev = c.seg;
     }
-    const int s = k % kStages;
-    const uint32_t ph = (k / kStages) & 1;
-    const int a = k & 1;
-    if (!mbar_wait(&b.qfull[s], ph, status, 0x1310u | s)) break;
     if (!mbar_wait(&b.qrelu[s], ph, status, 0x1320u | s)) break;
     if (!mbar_wait(&b.acce[a], ((k >> 1) & 1) ^ 1, status, 0x1330u | a)) break;
     tc_fence_after();
@@ -458,23 +503,24 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long lon
     }
     mma_commit(&b.qempty[s]);
     mma_commit(&b.accf[a]);
-    if (c.last || t == te - 1) mma_commit(&b.bempty[bb]);
   }
   mma_commit(b.done);
   mbar_wait(b.done, 0, status, 0x13F0u);
 }
 
-// ReLU of Q tile k (stage k % kStages) in place; returns false if the grid failed.
-__device__ __forceinline__ bool relu_q(uint8_t* smem, const Bars& b, long long k, bool two_atoms, int r, int lane,
-                                       uint32_t* status) {
+// ReLU of the k-th Q tile (stage k % kStages) in place. Returns 1 when done, 0 at the end of the
+// sequence, -1 if the grid failed.
+__device__ __forceinline__ int relu_q(uint8_t* smem, const Bars& b, const Seq& sq, long long k, bool two_atoms, int r,
+                                      int lane, uint32_t* status) {
   const int s = static_cast<int>(k % kStages);
   const bool ok = mbar_wait(&b.qfull[s], static_cast<uint32_t>((k / kStages) & 1), status, 0x1200u | s);
-  if (!warp_all(ok)) return false;
+  if (!warp_all(ok)) return -1;
+  if (sq.ring[k % kRing] < 0) return 0;
   relu_tile_inplace(smem + s * kQBytes, (two_atoms ? kQBytes : kAtomBytes) / 16, r);
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) mbar_arrive(&b.qrelu[s]);
-  return true;
+  return 1;
 }
 
 // Output staging: nbuf (1 or 2) sets of 4 warps x two 4 KB atoms starting at `base`.
@@ -487,13 +533,16 @@ struct Staging {
 // output columns 64h..64h+63; numerator times 1 / (denominator + eps), bf16, into this warp's
 // swizzled 4 KB staging atom (alternating between buffers when there are two), then a TMA store
 // clipped to the block.
-__device__ __forceinline__ bool epilogue_tile(const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo,
-                                              long long t, long long k, uint32_t tmem, int q, int h, int lane,
-                                              float eps, uint32_t* status) {
-  const TileCoord c = tile_coord(t, geo);
+// Returns 1 when done, 0 at the end of the sequence, -1 if the grid failed.
+__device__ __forceinline__ int epilogue_tile(const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo,
+                                             const Seq& sq, long long k, uint32_t tmem, int q, int h, int lane,
+                                             float eps, uint32_t* status) {
   const int a = static_cast<int>(k & 1);
   const bool ok = mbar_wait(&b.accf[a], static_cast<uint32_t>((k >> 1) & 1), status, 0x1400u | a);
-  if (!warp_all(ok)) return false;
+  if (!warp_all(ok)) return -1;
+  const long long t = sq.ring[k % kRing];
+  if (t < 0) return 0;
+  const TileCoord c = tile_coord(t, geo);
   tc_fence_after();
   const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
   uint32_t dr;
@@ -538,15 +587,14 @@ __device__ __forceinline__ bool epilogue_tile(const Staging& sg, const Bars& b, 
     }
     bulk_commit();  // one group per tile (possibly empty), so "all but the latest" means the previous tile
   }
-  return true;
+  return 1;
 }
 
 // Warps 0-3: epilogue of output columns 0..63 of every tile.
-__device__ void epilogue_role(const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo, long long tb,
-                              long long te, uint32_t tmem, int warp, int lane, float eps, uint32_t* status) {
-  long long k = 0;
-  for (long long t = tb; t < te; ++t, ++k)
-    if (!epilogue_tile(sg, b, m, geo, t, k, tmem, warp & 3, 0, lane, eps, status)) break;
+__device__ void epilogue_role(const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo, const Seq& sq,
+                              uint32_t tmem, int warp, int lane, float eps, uint32_t* status) {
+  for (long long k = 0;; ++k)
+    if (epilogue_tile(sg, b, m, geo, sq, k, tmem, warp & 3, 0, lane, eps, status) <= 0) break;
   if (lane == 0) bulk_wait_all();
 }
 
@@ -555,16 +603,24 @@ __device__ void epilogue_role(const Staging& sg, const Bars& b, const Maps4& m, 
 // after the epilogue of tile k: its stage was freed by the MMAs of tile k, which the epilogue has
 // waited for, so the order cannot deadlock.
 __device__ void relu_epi_role(uint8_t* smem, const Staging& sg, const Bars& b, const Maps4& m, const Geom& geo,
-                              long long tb, long long te, int relu_done, bool two_atoms, uint32_t tmem, int warp,
-                              int lane, float eps, uint32_t* status) {
+                              const Seq& sq, int relu_done, bool two_atoms, uint32_t tmem, int warp, int lane,
+                              float eps, uint32_t* status) {
   const int r = static_cast<int>(threadIdx.x) - 128;
-  const long long n = te - tb;
   long long kr = relu_done;  // tiles [0, relu_done) were ReLU'd by the caller
-  bool ok = true;
-  for (; kr < n && kr < kStages && ok; ++kr) ok = relu_q(smem, b, kr, two_atoms, r, lane, status);
-  for (long long k = 0; k < n && ok; ++k) {
-    if (two_atoms) ok = epilogue_tile(sg, b, m, geo, tb + k, k, tmem, warp & 3, 1, lane, eps, status);
-    if (ok && kr < n) ok = relu_q(smem, b, kr++, two_atoms, r, lane, status);
+  int rs = 1;                // relu state: 1 more tiles, 0 sequence ended, -1 failed
+  for (; kr < kStages && rs > 0; ++kr) rs = relu_q(smem, b, sq, kr, two_atoms, r, lane, status);
+  if (rs < 0) return;
+  for (long long k = 0;; ++k) {
+    if (two_atoms) {
+      const int es = epilogue_tile(sg, b, m, geo, sq, k, tmem, warp & 3, 1, lane, eps, status);
+      if (es <= 0) break;
+    } else if (rs == 0) {
+      break;
+    }
+    if (rs > 0) {
+      rs = relu_q(smem, b, sq, kr++, two_atoms, r, lane, status);
+      if (rs < 0) break;
+    }
   }
   if (two_atoms && lane == 0) bulk_wait_all();
 }
@@ -648,11 +704,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + ot::kRegionBytes);
   const ot::Bars b = ot::bars_at(barmem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + ot::kNumBars);
+  volatile long long* ring = reinterpret_cast<volatile long long*>(barmem + ot::kNumBars + 1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
-  const long long tb = tile_begin(g, geo);
-  const long long te = tile_begin(g + 1, geo);
+  // static range of this CTA, then chunks of the dynamic tail (counter reset by the scan kernel)
+  const ot::Seq sq{out_tile_begin(g, geo), out_tile_begin(g + 1, geo), geo.T - geo.tdyn, geo.T,
+                   geo.tdyn > 0 ? status + 6 : nullptr, ring};
   const bool two_atoms = geo.D > 64;
   const Maps4 m{&q_main, &q_last, &o_main, &o_last};
   if (threadIdx.x == 0) {
@@ -664,17 +722,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == kWarpProducer) {
     if (lane == 0) {
-      const int pre = ot::prefill(smem, b, m, geo, tb, te, two_atoms);
-      griddep_wait();  // the prefix tiles come from the scan grid
-      ot::produce(smem, b, m, geo, tb, te, pre, two_atoms, ptiles, nullptr, 0, status);
+      const int pre = ot::prefill(smem, b, m, geo, sq, two_atoms);
+      griddep_wait();  // the prefix tiles and the chunk counter come from the scan grid
+      ot::produce(smem, b, m, geo, sq, pre, two_atoms, ptiles, nullptr, 0, status);
     }
   } else if (warp >= 4 && warp < 8) {
-    ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, m, geo, tb, te, 0, two_atoms, tmem, warp, lane,
-                      eps, status);
+    ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, 0, two_atoms, tmem, warp, lane, eps,
+                      status);
   } else if (warp == kWarpMma) {
-    if (lane == 0) ot::mma_role(smem, b, geo, tb, te, two_atoms, tmem, status);
+    if (lane == 0) ot::mma_role(smem, b, geo, sq, two_atoms, tmem, status);
   } else {
-    ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, b, m, geo, tb, te, tmem, warp, lane, eps, status);
+    ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, tmem, warp, lane, eps, status);
   }
   persistent_teardown(tmem, warp);
 }
@@ -710,8 +768,12 @@ __global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ pa
                                                     const int2* __restrict__ segcta, const Geom geo,
                                                     const float* S_in, const float* z_in, float* S_out,
                                                     float* z_out, uint8_t* __restrict__ ptiles,
-                                                    float* __restrict__ p32, const int ng_warps) {
+                                                    float* __restrict__ p32, const int ng_warps,
+                                                    uint32_t* out_chunks) {
   griddep_wait();  // partials come from the state kernel; prefix tiles may still be read before it
+  // The output kernel of this call claims its dynamic chunks from this counter only after this
+  // grid has completed; the previous call's output kernel completed before the state kernel did.
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *out_chunks = 0u;
   griddep_launch_dependents();
   // block (bh, rows e = blockIdx.y * R .. + R - 1): warp w handles row r = w / ng, block group j = w % ng
   extern __shared__ float4 s_scan[];   // [R][ng][32] warp totals, then [R][32] incoming cache
@@ -1029,6 +1091,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
   uint64_t* flushed = barmem + st::kNumBars + ot::kNumBars;  // epilogue warps finished a slot (count 4)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flushed + 1);
+  volatile long long* ring = reinterpret_cast<volatile long long*>(flushed + 2);
   uint64_t* seqp = reinterpret_cast<uint64_t*>(status + 2);  // header bytes 8..15: launch sequence number
   uint32_t* gstart = status + 4;                             // header bytes 16..19: CTAs that read the tag
   const int warp = threadIdx.x >> 5;
@@ -1091,7 +1154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // phase 2: the Q stages fill (Q does not depend on the state, and the stages are free once the
   // state MMAs retired) while the CTA takes its share of the combine of its head(s): whole prefix
   // rows, so each cache element belongs to exactly one CTA.
-  if (warp == kWarpProducer && lane == 0) pre = ot::prefill(smem, ob, mqo, geo, tb, te, two_atoms);
+  const ot::Seq sq{tb, te, 0, 0, nullptr, ring};
+  if (warp == kWarpProducer && lane == 0) pre = ot::prefill(smem, ob, mqo, geo, sq, two_atoms);
   float* sS = reinterpret_cast<float*>(smem + fu::kScratchOff);
   float* sZ = reinterpret_cast<float*>(smem + fu::kScratchZOff);
   const int h0 = tile_coord(tb, geo).seg;
@@ -1121,14 +1185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // phase 3: output of the same tiles, each head as soon as its combine is complete
   if (s_ok) {
     if (warp == kWarpProducer) {
-      if (lane == 0) ot::produce(smem, ob, mqo, geo, tb, te, pre, two_atoms, ptiles, combined, tag, status);
+      if (lane == 0) ot::produce(smem, ob, mqo, geo, sq, pre, two_atoms, ptiles, combined, tag, status);
     } else if (warp >= 4 && warp < 8) {
-      ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, ob, mqo, geo, tb, te, 0, two_atoms, tmem, warp, lane,
+      ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, ob, mqo, geo, sq, 0, two_atoms, tmem, warp, lane,
                         eps, status);
     } else if (warp == kWarpMma) {
-      if (lane == 0) ot::mma_role(smem, ob, geo, tb, te, two_atoms, tmem, status);
+      if (lane == 0) ot::mma_role(smem, ob, geo, sq, two_atoms, tmem, status);
     } else {
-      ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, ob, mqo, geo, tb, te, tmem, warp, lane, eps, status);
+      ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, ob, mqo, geo, sq, tmem, warp, lane, eps, status);
     }
   } else if (warp == kWarpProducer && lane == 0) {
     for (int i = 0; i < pre; ++i) mbar_wait(&ob.qfull[i], 0, status, 0x2180u);  // prefilled loads land
@@ -1272,6 +1336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const st::Bars sb = st::bars_at(barmem);
   const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + st::kNumBars + ot::kNumBars);
+  volatile long long* ring = reinterpret_cast<volatile long long*>(barmem + st::kNumBars + ot::kNumBars + 1);
   float* part = reinterpret_cast<float*>(smem + cl::kPartOff);
   float* sS = reinterpret_cast<float*>(smem + cl::kScratchOff);
   float* sZ = reinterpret_cast<float*>(smem + cl::kScratchZOff);
@@ -1316,16 +1381,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   // phase 2: Q stages fill while the cluster exchanges the partial states. The Q loads are issued
   // after the first cluster barrier: issued before it, they delayed its release by about 1 us.
   const int pre = static_cast<int>(te - tb < ot::kStages ? te - tb : ot::kStages);  // Q tiles prefilled
+  const ot::Seq sq{tb, te, 0, 0, nullptr, ring};
   cluster_arrive_release();
   cluster_wait_acquire();
-  if (warp == kWarpProducer && lane == 0) ot::prefill(smem, ob, mqo, geo, tb, te, two_atoms);
+  if (warp == kWarpProducer && lane == 0) ot::prefill(smem, ob, mqo, geo, sq, two_atoms);
   // The ReLU warps rewrite the prefilled Q tiles that have already landed while the other warps
   // combine (the combine is bound by distributed-shared-memory bandwidth, not by its thread count);
   // tiles still in flight are left to phase 3 so that the second barrier never waits for Q.
   int relu_done = 0;
   if (warp >= 4 && warp < 8) {
     while (relu_done < pre && warp_all(mbar_try_wait(&ob.qfull[relu_done], 0)) &&
-           ot::relu_q(smem, ob, relu_done, two_atoms, threadIdx.x - 128, lane, status))
+           ot::relu_q(smem, ob, sq, relu_done, two_atoms, threadIdx.x - 128, lane, status) > 0)
       ++relu_done;
   } else {
     const int tid = warp < 4 ? static_cast<int>(threadIdx.x) : 128 + (warp - kWarpProducer) * 32 + lane;
@@ -1343,13 +1409,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // failed wait anywhere in the grid every later wait returns at once, so phase 3 runs regardless.)
   const ot::Staging sg{smem + cl::kPartOff, 2};
   if (warp == kWarpProducer) {
-    if (lane == 0) ot::produce(smem, ob, mqo, geo, tb, te, pre, two_atoms, nullptr, nullptr, 0, status);
+    if (lane == 0) ot::produce(smem, ob, mqo, geo, sq, pre, two_atoms, nullptr, nullptr, 0, status);
   } else if (warp >= 4 && warp < 8) {
-    ot::relu_epi_role(smem, sg, ob, mqo, geo, tb, te, relu_done, two_atoms, tmem, warp, lane, eps, status);
+    ot::relu_epi_role(smem, sg, ob, mqo, geo, sq, relu_done, two_atoms, tmem, warp, lane, eps, status);
   } else if (warp == kWarpMma) {
-    if (lane == 0) ot::mma_role(smem, ob, geo, tb, te, two_atoms, tmem, status);
+    if (lane == 0) ot::mma_role(smem, ob, geo, sq, two_atoms, tmem, status);
   } else {
-    ot::epilogue_role(sg, ob, mqo, geo, tb, te, tmem, warp, lane, eps, status);
+    ot::epilogue_role(sg, ob, mqo, geo, sq, tmem, warp, lane, eps, status);
   }
   // the outgoing cache last: nothing in this launch reads it, and its stores drain with the output
   // (lanes 1..31 of the producer and MMA warps wait for lane 0 first, so they do not compete with it)
@@ -1624,7 +1690,8 @@ cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const Bl
 }
 
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
-                        float* S_out, float* z_out, void* ptiles_bf16, float* p32, cudaStream_t s) {
+                        float* S_out, float* z_out, void* ptiles_bf16, float* p32, uint32_t* out_chunks,
+                        cudaStream_t s) {
   // ng warps share the blocks of one row; R rows per block so that a block has up to 16 warps
   int ng = (g.nblk + kScanReg - 1) / kScanReg;
   if (ng > kScanMaxWarps) ng = kScanMaxWarps;
@@ -1633,7 +1700,7 @@ cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g
   while (R > 1 && (R * ng > 16 || kPTileRows % R != 0)) R >>= 1;
   const size_t smem = static_cast<size_t>(R) * (ng + 1) * 32 * sizeof(float4);
   return launch_pdl(scan_kernel, dim3(g.BH, kPTileRows / R), dim3(32 * ng * R), smem, s, partials, segcta, g, S_in,
-                    z_in, S_out, z_out, static_cast<uint8_t*>(ptiles_bf16), p32, ng);
+                    z_in, S_out, z_out, static_cast<uint8_t*>(ptiles_bf16), p32, ng, out_chunks);
 }
 
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,

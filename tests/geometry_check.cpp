@@ -5,7 +5,9 @@
 //  - the CTA interval [cta_of(first), cta_of(last)] of each segment is exactly the set of CTAs
 //    that flush a partial for it,
 //  - with one block per head, the CTAs sharing a head's combine [ga, gb] form a non-empty
-//    sub-interval of the CTAs covering it, so their flags (index g + h) are unique slots.
+//    sub-interval of the CTAs covering it, so their flags (index g + h) are unique slots,
+//  - the output pass's static ranges tile [0, T - tdyn) exactly, every CTA keeps at least 3 static
+//    tiles when there is a dynamic tail, and the tail is a whole number of chunks.
 #include <cstdio>
 #include <cstdlib>
 #include <set>
@@ -41,6 +43,12 @@ static int check(int B, int H, int N, int L, int sms) {
   }
   for (size_t i = 0; i < covered.size(); ++i)
     if (covered[i] != 1) { printf("token %zu covered %d times\n", i, covered[i]); return 1; }
+  if (g.tdyn < 0 || g.tdyn % kOutChunk != 0 || g.tdyn >= g.T) { printf("tdyn %lld\n", g.tdyn); return 1; }
+  if (out_tile_begin(0, g) != 0 || out_tile_begin(g.G, g) != g.T - g.tdyn) { printf("output ranges\n"); return 1; }
+  for (int cta = 0; cta < g.G; ++cta) {
+    const long long n = out_tile_begin(cta + 1, g) - out_tile_begin(cta, g);
+    if (n < 1 || (g.tdyn > 0 && n < 3)) { printf("output static range of cta %d: %lld tiles\n", cta, n); return 1; }
+  }
   for (int s = 0; s < g.nseg; ++s) {
     long long f = seg_first_tile(s, g);
     int g0 = cta_of_tile(f, g), g1 = cta_of_tile(f + seg_ntiles(s, g) - 1, g);
