@@ -744,8 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // e = 129..143 are the zero rows of the bf16 B operand. Lane q owns key features 4q..4q+3;
 // warp j owns blocks [j*nblk/ng, (j+1)*nblk/ng) (at most kScanReg of them when nblk <= 128),
 // so every partial load is independent; the running prefix crosses warps through shared memory.
-constexpr int kScanReg = 4;
-constexpr int kScanMaxWarps = 32;
+constexpr int kScanReg = 8;
+constexpr int kScanMaxWarps = 16;
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
@@ -764,7 +764,7 @@ __device__ __forceinline__ float4 block_sum(const float* __restrict__ partials, 
   return acc;
 }
 
-__global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ partials,
+__global__ void __launch_bounds__(512) scan_kernel(const float* __restrict__ partials,
                                                     const int2* __restrict__ segcta, const Geom geo,
                                                     const float* S_in, const float* z_in, float* S_out,
                                                     float* z_out, uint8_t* __restrict__ ptiles,
@@ -796,16 +796,33 @@ __global__ void __launch_bounds__(1024) scan_kernel(const float* __restrict__ pa
   const bool live = e < kPartRows;
   const int seg0 = bh * nblk;
 
-  // pass 1: this warp's block sums (kept in registers) and their total
+  // pass 1: this warp's block sums (kept in registers) and their total. The slot ranges of all
+  // kScanReg blocks are fetched together, then the first two slots of every block together (a
+  // block of a long sequence is rarely covered by more than two CTAs; further slots follow), so
+  // the warp waits for two memory round trips instead of two per block.
   float4 sums[kScanReg];
   float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+  int2 gr[kScanReg];
+#pragma unroll
+  for (int i = 0; i < kScanReg; ++i) gr[i] = (live && i < cnt) ? segcta[seg0 + c0 + i] : make_int2(0, -1);
+  float4 p0[kScanReg], p1[kScanReg];
 #pragma unroll
   for (int i = 0; i < kScanReg; ++i) {
-    sums[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (live && i < cnt) {
-      sums[i] = block_sum(partials, segcta, seg0 + c0 + i, e, d0);
-      tot = f4add(tot, sums[i]);
-    }
+    const size_t row = static_cast<size_t>(seg0 + c0 + i) * kPartRows + e;
+    p0[i] = gr[i].y >= gr[i].x ? __ldcg(reinterpret_cast<const float4*>(
+                                     partials + (static_cast<size_t>(gr[i].x) * kPartRows + row) * kDPad + d0))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    p1[i] = gr[i].y >= gr[i].x + 1 ? __ldcg(reinterpret_cast<const float4*>(
+                                         partials + (static_cast<size_t>(gr[i].x + 1) * kPartRows + row) * kDPad + d0))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < kScanReg; ++i) {
+    sums[i] = f4add(p0[i], p1[i]);
+    for (int gg = gr[i].x + 2; gg <= gr[i].y; ++gg)
+      sums[i] = f4add(sums[i], __ldcg(reinterpret_cast<const float4*>(
+                                   partials + (static_cast<size_t>(gg + seg0 + c0 + i) * kPartRows + e) * kDPad + d0)));
+    tot = f4add(tot, sums[i]);
   }
   for (int i = kScanReg; i < cnt; ++i)
     if (live) tot = f4add(tot, block_sum(partials, segcta, seg0 + c0 + i, e, d0));
@@ -1692,12 +1709,13 @@ cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const Bl
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
                         float* S_out, float* z_out, void* ptiles_bf16, float* p32, uint32_t* out_chunks,
                         cudaStream_t s) {
-  // ng warps share the blocks of one row; R rows per block so that a block has up to 16 warps
+  // ng warps share the blocks of one row (kScanReg each in registers); R rows per block so that a
+  // block has a few warps: at ~124 registers per thread, small blocks pack the SMs best.
   int ng = (g.nblk + kScanReg - 1) / kScanReg;
   if (ng > kScanMaxWarps) ng = kScanMaxWarps;
   if (ng < 1) ng = 1;
-  int R = 16;
-  while (R > 1 && (R * ng > 16 || kPTileRows % R != 0)) R >>= 1;
+  int R = 4;
+  while (R > 1 && (R * ng > 4 || kPTileRows % R != 0)) R >>= 1;
   const size_t smem = static_cast<size_t>(R) * (ng + 1) * 32 * sizeof(float4);
   return launch_pdl(scan_kernel, dim3(g.BH, kPTileRows / R), dim3(32 * ng * R), smem, s, partials, segcta, g, S_in,
                     z_in, S_out, z_out, static_cast<uint8_t*>(ptiles_bf16), p32, ng, out_chunks);
