@@ -10,6 +10,12 @@
 
 namespace sv {
 
+// Workspace header (the first kHeaderBytes of every workspace, zeroed by sv_workspace_init):
+//   bytes  0..3   status word: 0, or kDevTimeout | site of the first bounded wait that expired
+//   bytes  8..15  launch sequence number of the one-block kernel (its flags carry it)
+//   bytes 16..19  CTAs of the current one-block launch that have read the sequence number
+//   bytes 24..27  dynamic output-chunk counter of the output kernel (reset by the scan kernel)
+
 // Tensor maps of one [BH, N, D] bf16 tensor seen as blocks: `main` covers the blocks of length L,
 // `last` the shorter last block when N is not a multiple of L (else it repeats `main`).
 struct BlockMaps {
