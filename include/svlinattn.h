@@ -78,7 +78,8 @@ typedef struct CUstream_st* sv_stream_t; /* same type as cudaStream_t */
  * SV_OP_BLOCK_CAUSAL_ATTN. Returns 0 for invalid sizes (see sv_last_error). */
 size_t sv_workspace_bytes(sv_op op, int B, int H, int N, int D, int block_len, sv_dtype dt);
 
-/* Zero the workspace's status word (asynchronous on `stream`). Call once after allocating. */
+/* Zero the whole workspace (asynchronous on `stream`): the status word, the launch sequence words
+ * and the flags between CTAs all start at zero. Call once after allocating. */
 sv_status sv_workspace_init(void* ws, size_t ws_bytes, sv_stream_t stream);
 
 /* Synchronise `stream`, read the workspace's status word and clear it. SV_OK if no kernel
@@ -128,9 +129,9 @@ sv_status sv_cache_step(const void* q, const void* k, const void* v, void* o, in
  * sv_cache_step. A call that needs more scratch than 16 MiB (see sv_workspace_bytes with
  * SV_OP_CACHE_STEP: about 66 KB per (batch, head) pair plus 66 KB per streaming multiprocessor,
  * so the 720p streaming block [1, 20, 2760, 128] needs about 12 MB and B * H above ~100 does not
- * fit) is refused with SV_ERR_INVALID_ARG before any launch. All calls on a device share the array: calls that may
- * overlap on the GPU race. The first call on a device looks up the array's device address; make
- * it before any stream capture. Device-side wait timeouts are not reported through this entry
+ * fit) is refused with SV_ERR_INVALID_ARG before any launch. All calls on a device share the
+ * array: calls that may overlap on the GPU race. The first call on a device looks up the array's
+ * device address; make it before any stream capture. Device-side wait timeouts are not reported through this entry
  * point (use sv_cache_step with a workspace and sv_device_status for that). */
 sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
                                 sv_dtype dt, float eps, float* S, float* z, int commit, sv_stream_t stream);
@@ -139,13 +140,14 @@ sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, voi
  * the caller), the calling thread's following forward calls (sv_linattn_fwd, sv_block_causal_attn,
  * sv_cache_step) record events[0] before the state-reduction kernel, events[1] after it,
  * events[2] after the prefix scan and events[3] after the output kernel, on the call's stream.
+ * When a call runs as a single launch (bf16, one block per head) events[1..3] all follow it.
+ * Events between the kernels keep them from overlapping, so time with the hook removed.
  * events == NULL (n ignored) removes the hook. Costs one cudaEventRecord per mark. */
 sv_status sv_profile_events(void* const* events, int n);
 
 /* Message for the calling thread's most recent non-OK status ("" if none). */
 const char* sv_last_error(void);
 
-/* Library version, major * 10000 + minor * 100 + patch. */
 /* Failure-path self-test of the kernels' bounded waits; makes no GPU fault and leaves nothing in
  * flight. Launches one CTA whose waiters block, through the same bounded-wait routine the pipeline
  * kernels use, on an mbarrier phase that nothing completes. After the wait limit (about 2 s) the
@@ -156,6 +158,7 @@ const char* sv_last_error(void);
  * read afterwards with sv_device_status, which then returns SV_ERR_TIMEOUT and clears the word. */
 sv_status sv_selftest_wait_timeout(void* ws, size_t ws_bytes, sv_stream_t stream);
 
+/* Library version, major * 10000 + minor * 100 + patch. */
 int sv_version(void);
 
 #ifdef __cplusplus
