@@ -156,8 +156,10 @@ sv_status check_sizes(int B, int H, int N, int D, int block_len, sv_dtype dt) {
   if (N < 1) return fail(SV_ERR_INVALID_ARG, "N=%d must be >= 1", N);
   if (block_len < 1) return fail(SV_ERR_INVALID_ARG, "block_len=%d must be >= 1", block_len);
   if (dt == SV_BF16) {
-    if (D < 64 || D > 128 || D % 16 != 0)
-      return fail(SV_ERR_UNSUPPORTED, "bf16 path needs D in {64, 80, 96, 112, 128}, got D=%d", D);
+    // rows of D bf16 values must be a whole number of 16-byte units for the TMA tensor maps; features
+    // beyond D inside the 64-wide tile columns are zero-filled on load and clipped on store
+    if (D < 8 || D > 128 || D % 8 != 0)
+      return fail(SV_ERR_UNSUPPORTED, "bf16 path needs D a multiple of 8 in [8, 128], got D=%d", D);
   } else if (D < 1 || D > 128) {
     return fail(SV_ERR_UNSUPPORTED, "fp32 path needs 1 <= D <= 128, got D=%d", D);
   }

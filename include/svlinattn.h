@@ -28,8 +28,8 @@
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *    Pointers stay owned by the caller; the library allocates nothing and keeps no state
  *    between calls other than per-device kernel attributes.
- *  - Supported sizes: B, H, N >= 1; SV_BF16: D in {64, 80, 96, 112, 128};
- *    SV_F32: 1 <= D <= 128. eps must be finite and >= 0.
+ *  - Supported sizes: B, H, N >= 1; SV_BF16: D a multiple of 8 in [8, 128] (a row must be a whole
+ *    number of 16-byte units); SV_F32: 1 <= D <= 128. eps must be finite and >= 0.
  *  - Errors: every argument is checked on the host BEFORE anything is launched; a bad argument
  *    returns SV_ERR_INVALID_ARG / SV_ERR_UNSUPPORTED and launches nothing. A failed launch returns
  *    SV_ERR_CUDA. Device-side timeouts (SV_ERR_TIMEOUT) are reported by sv_device_status.

@@ -95,6 +95,11 @@ def test_fp32_shapes(sv, B, H, N, D, L):
     (1, 2, 5, 128, 1),         # block_len = 1: token-causal
     (1, 1, 257, 128, 1000),    # block_len > N
     (3, 5, 333, 128, 111),
+    (1, 2, 600, 32, 256),      # D = 32 (half a feature atom, zero-filled), as config 0 but bf16
+    (1, 2, 450, 48, 100),      # D = 48
+    (2, 1, 300, 8, 77),        # D = 8: a 16-byte row
+    (1, 2, 400, 72, 150),      # D = 72 (second atom holds 8 features)
+    (1, 1, 260, 120, 260),     # D = 120, bidirectional
 ])
 def test_bf16_shapes(sv, B, H, N, D, L):
     st, (q, k, v) = inputs((B, H, N, D), 1, "bf16")
@@ -120,7 +125,8 @@ def test_bf16_many_tiles_per_cta(sv):
 # the partial states through distributed shared memory; incoming cache, in-place update
 # --------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("B,H,N,D", [(1, 20, 800, 128), (2, 10, 2760, 128), (1, 24, 1000, 112),
-                                     (1, 20, 1500, 64), (1, 20, 700, 96)])
+                                     (1, 20, 1500, 64), (1, 20, 700, 96), (1, 20, 900, 32),
+                                     (1, 16, 1200, 40)])
 def test_one_block_few_heads_with_cache(sv, B, H, N, D):
     st, (q, k, v) = inputs((B, H, N, D), 5, "bf16")
     g = np.random.default_rng(7)
@@ -144,9 +150,9 @@ def test_bf16_error_is_well_inside_tolerance(sv):
     assert err < 5e-3, err
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_incoming_cache_and_in_place_update(sv, dtype):
-    B, H, N, D, L = 1, 3, 600, 128, 250
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 128), ("bf16", 48)])
+def test_incoming_cache_and_in_place_update(sv, dtype, D):
+    B, H, N, L = 1, 3, 600, 250
     st, (q, k, v) = inputs((B, H, N, D), 4, dtype)
     rng = np.random.default_rng(4)
     S0 = rng.standard_normal((B, H, D, D)).astype(np.float32) * 30
@@ -160,9 +166,9 @@ def test_incoming_cache_and_in_place_update(sv, dtype):
     assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_state_update(sv, dtype):
-    B, H, N, D = 2, 2, 777, 128
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 128), ("bf16", 32), ("bf16", 88)])
+def test_state_update(sv, dtype, D):
+    B, H, N = 2, 2, 777
     st, (_, k, v) = inputs((B, H, N, D), 6, dtype)
     rng = np.random.default_rng(6)
     S0 = rng.standard_normal((B, H, D, D)).astype(np.float32)

@@ -55,7 +55,8 @@ def test_validation_rejects_before_any_launch(lib):
     assert b"q is NULL" in lib.sv_last_error()
     assert f(fake, fake, fake, fake, 1, 1, 0, 128, 0, 1e-6, fake, 1 << 30, None) == 1      # N = 0
     assert f(fake, fake, fake, fake, 1, 1, 128, 100, 0, 1e-6, fake, 1 << 30, None) == 2    # bf16 D=100
-    assert f(fake, fake, fake, fake, 1, 1, 128, 32, 0, 1e-6, fake, 1 << 30, None) == 2     # bf16 D=32
+    assert f(fake, fake, fake, fake, 1, 1, 128, 36, 0, 1e-6, fake, 1 << 30, None) == 2     # bf16 D=36
+    assert f(fake, fake, fake, fake, 1, 1, 128, 136, 0, 1e-6, fake, 1 << 30, None) == 2    # bf16 D>128
     assert f(fake, fake, fake, fake, 1, 1, 128, 129, 1, 1e-6, fake, 1 << 30, None) == 2    # f32 D>128
     assert f(fake, fake, fake, fake, 1, 1, 128, 128, 7, 1e-6, fake, 1 << 30, None) == 2    # dtype
     assert f(fake, vp(256 * 1024 + 2), fake, fake, 1, 1, 128, 128, 0, 1e-6, fake, 1 << 30, None) == 1  # misaligned
