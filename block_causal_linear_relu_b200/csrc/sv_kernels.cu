@@ -362,9 +362,8 @@ __device__ __forceinline__ void init_bars(const Bars& b, bool two_atoms) {
   mbar_init(b.done, 1);
 }
 
-__device__ __forceinline__ void load_q(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo, long long t,
-                                       int s, bool two_atoms, uint64_t pol) {
-  const TileCoord c = tile_coord(t, geo);
+__device__ __forceinline__ void load_q(uint8_t* smem, const Bars& b, const Maps4& m, const Geom& geo,
+                                       const TileCoord& c, int s, bool two_atoms, uint64_t pol) {
   const bool lst = use_last_map(c, geo);
   const CUtensorMap* mq = lst ? m.a_last : m.a_main;
   const int cb = lst ? 0 : c.blk;
@@ -377,16 +376,30 @@ __device__ __forceinline__ void load_q(uint8_t* smem, const Bars& b, const Maps4
 // The output tiles of a CTA: its static range [tb, te), then, when `counter` is set, chunks of
 // kDynChunk tiles of [dyn_begin, dyn_end) claimed through an atomic counter by whichever CTA gets
 // there first (output tiles are independent, so the result does not depend on who computes what).
-// The producer walks the sequence and writes the k-th tile's index into ring[k % kRing] before
-// the barrier the other roles wait on for that tile (qfull); -1 ends the sequence.
+// The producer walks the sequence and writes the k-th tile's coordinates into ring[k % kRing]
+// (x = segment, y = (batch, head), z = block, w = first token in the block) before the barrier the
+// other roles wait on for that tile (qfull); x = -1 ends the sequence. The MMA and epilogue loops
+// thus do no index arithmetic of their own: on one thread a tile's coordinates cost a 64-bit
+// division chain, which sat on the critical path of short sequences.
+// An entry is rewritten (tile k + kRing) only after the MMAs of tile k + kRing - kStages retired,
+// by which time every role has read entry k.
 constexpr int kRing = 8;
 constexpr int kDynChunk = kOutChunk;
+constexpr int kRingBytes = kRing * 16;
 struct Seq {
   long long tb, te;
   long long dyn_begin, dyn_end;
   uint32_t* counter;
-  volatile long long* ring;
+  volatile int4* ring;
 };
+__device__ __forceinline__ void ring_put(const Seq& sq, int k, const TileCoord& c) {
+  volatile int4* e = sq.ring + (k % kRing);
+  e->y = c.bh;
+  e->z = c.blk;
+  e->w = c.tok0;
+  e->x = c.seg;
+}
+__device__ __forceinline__ void ring_end(const Seq& sq, int k) { sq.ring[k % kRing].x = -1; }
 
 // Q was final before the state reduction ran, so the first stages of the static range can fill
 // before the prefix exists. Returns how many tiles were issued.
@@ -394,8 +407,9 @@ __device__ int prefill(uint8_t* smem, const Bars& b, const Maps4& m, const Geom&
   const uint64_t pol = policy_evict_first();
   const int pre = static_cast<int>(sq.te - sq.tb < kStages ? sq.te - sq.tb : kStages);
   for (int i = 0; i < pre; ++i) {
-    sq.ring[i] = sq.tb + i;
-    load_q(smem, b, m, geo, sq.tb + i, i, two_atoms, pol);
+    const TileCoord c = tile_coord(sq.tb + i, geo);
+    ring_put(sq, i, c);
+    load_q(smem, b, m, geo, c, i, two_atoms, pol);
   }
   return pre;
 }
@@ -443,14 +457,14 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
     if (k >= pre) {
       const int s = k % kStages;
       if (!mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1120u | s)) { ok = false; break; }
-      sq.ring[k % kRing] = t;
-      load_q(smem, b, m, geo, t, s, two_atoms, pol);
+      ring_put(sq, k, c);
+      load_q(smem, b, m, geo, c, s, two_atoms, pol);
     }
   }
   if (ok) {  // end of the sequence: a plain arrival completes the next stage's qfull with index -1
     const int s = k % kStages;
     if (k < pre || mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1140u | s)) {
-      sq.ring[k % kRing] = -1;
+      ring_end(sq, k);
       mbar_arrive(&b.qfull[s]);
       ++k;
     }
@@ -470,8 +484,8 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, const Se
     const uint32_t ph = (k / kStages) & 1;
     const int a = k & 1;
     if (!mbar_wait(&b.qfull[s], ph, status, 0x1310u | s)) break;
-    const long long t = sq.ring[k % kRing];
-    if (t < 0) {
+    const int seg = sq.ring[k % kRing].x;
+    if (seg < 0) {
       // End of the sequence, announced on this accumulator's barrier under the same flow control
       // as a tile: first the epilogue must have released the accumulator's previous use (tile
       // k - 2), or the barrier could run two phases ahead of a slow epilogue, which would then
@@ -481,13 +495,12 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, const Se
       mma_commit(&b.accf[a]);
       break;
     }
-    const TileCoord c = tile_coord(t, geo);
-    if (c.seg != prev) {
+    if (seg != prev) {
       if (j > 0) mma_commit(&b.bempty[(j - 1) & 1]);  // the previous prefix tile is free once its MMAs retire
       bb = j & 1;
       if (!mbar_wait(&b.bfull[bb], (j >> 1) & 1, status, 0x1300u | bb)) break;
       ++j;
-      prev = c.seg;
+      prev = seg;
     }
     if (!mbar_wait(&b.qrelu[s], ph, status, 0x1320u | s)) break;
     if (!mbar_wait(&b.acce[a], ((k >> 1) & 1) ^ 1, status, 0x1330u | a)) break;
@@ -515,7 +528,7 @@ __device__ __forceinline__ int relu_q(uint8_t* smem, const Bars& b, const Seq& s
   const int s = static_cast<int>(k % kStages);
   const bool ok = mbar_wait(&b.qfull[s], static_cast<uint32_t>((k / kStages) & 1), status, 0x1200u | s);
   if (!warp_all(ok)) return -1;
-  if (sq.ring[k % kRing] < 0) return 0;
+  if (sq.ring[k % kRing].x < 0) return 0;
   relu_tile_inplace(smem + s * kQBytes, (two_atoms ? kQBytes : kAtomBytes) / 16, r);
   fence_proxy_async_smem();
   __syncwarp();
@@ -540,9 +553,8 @@ __device__ __forceinline__ int epilogue_tile(const Staging& sg, const Bars& b, c
   const int a = static_cast<int>(k & 1);
   const bool ok = mbar_wait(&b.accf[a], static_cast<uint32_t>((k >> 1) & 1), status, 0x1400u | a);
   if (!warp_all(ok)) return -1;
-  const long long t = sq.ring[k % kRing];
-  if (t < 0) return 0;
-  const TileCoord c = tile_coord(t, geo);
+  const volatile int4* ent = sq.ring + (k % kRing);
+  if (ent->x < 0) return 0;
   tc_fence_after();
   const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
   uint32_t dr;
@@ -550,6 +562,7 @@ __device__ __forceinline__ int epilogue_tile(const Staging& sg, const Bars& b, c
   tmem_ld_x1(ta + kZRow, dr);
   tmem_ld_x32(ta + h * 64, rr[0]);
   tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+  const int bh = ent->y, blk = ent->z, tok0 = ent->w;  // read while the TMEM loads are in flight
   tmem_wait_ld();
   tc_fence_before();
   __syncwarp();
@@ -579,11 +592,12 @@ __device__ __forceinline__ int epilogue_tile(const Staging& sg, const Bars& b, c
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    const int blen = (c.blk == geo.nblk - 1) ? geo.Llast : geo.L;
-    const int row0 = c.tok0 + q * 32;
+    const bool in_last = blk == geo.nblk - 1;
+    const int blen = in_last ? geo.Llast : geo.L;
+    const int row0 = tok0 + q * 32;
     if (row0 < blen) {
-      const bool lst = use_last_map(c, geo);
-      tma_store_4d(lst ? m.b_last : m.b_main, ob, h * 64, row0, lst ? 0 : c.blk, c.bh);
+      const bool lst = in_last && geo.Llast != geo.L;  // the shorter last block has its own map
+      tma_store_4d(lst ? m.b_last : m.b_main, ob, h * 64, row0, lst ? 0 : blk, bh);
     }
     bulk_commit();  // one group per tile (possibly empty), so "all but the latest" means the previous tile
   }
@@ -656,7 +670,10 @@ __device__ __forceinline__ void persistent_teardown(uint32_t tmem, int warp) {
 // stand-alone kernels
 // ------------------------------------------------------------------------------------------
 constexpr int kStateSmem = st::kRegionBytes + 1024 + 256 + 1024;   // region, barriers, alignment slack
-constexpr int kOutSmem = ot::kRegionBytes + 1024 + 256 + 1024;
+constexpr int kOutSmem = ot::kRegionBytes + 1024 + 512 + 1024;
+// barrier areas (512 B): the barriers, the TMEM slot, then the 16-byte aligned tile ring
+static_assert((ot::kNumBars + 2) * 8 + ot::kRingBytes <= 512, "output kernel barrier area");
+static_assert((st::kNumBars + ot::kNumBars + 2) * 8 + ot::kRingBytes <= 512, "single-launch barrier area");
 
 __global__ void __launch_bounds__(kThreads, 1)
     state_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
@@ -704,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + ot::kRegionBytes);
   const ot::Bars b = ot::bars_at(barmem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + ot::kNumBars);
-  volatile long long* ring = reinterpret_cast<volatile long long*>(barmem + ot::kNumBars + 1);
+  volatile int4* ring = reinterpret_cast<volatile int4*>(barmem + ot::kNumBars + 2);  // 16-byte aligned
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -1108,7 +1125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
   uint64_t* flushed = barmem + st::kNumBars + ot::kNumBars;  // epilogue warps finished a slot (count 4)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flushed + 1);
-  volatile long long* ring = reinterpret_cast<volatile long long*>(flushed + 2);
+  volatile int4* ring = reinterpret_cast<volatile int4*>(flushed + 2);  // 16-byte aligned
   uint64_t* seqp = reinterpret_cast<uint64_t*>(status + 2);  // header bytes 8..15: launch sequence number
   uint32_t* gstart = status + 4;                             // header bytes 16..19: CTAs that read the tag
   const int warp = threadIdx.x >> 5;
@@ -1240,7 +1257,7 @@ static_assert(kPartOff + 2 * 4 * ot::kOWarpBytes <= fu::kRegion, "double-buffere
 constexpr int kShareRowsMax = (kPTileRows + kMinCluster - 1) / kMinCluster;
 constexpr int kScratchOff = fu::kRegion;                          // incoming-cache share, transposed
 constexpr int kScratchZOff = kScratchOff + kShareRowsMax * (kDPad + 1) * 4;
-constexpr int kBarOff = (kScratchZOff + kDPad * 4 + 7) / 8 * 8;
+constexpr int kBarOff = (kScratchZOff + kDPad * 4 + 127) / 128 * 128;
 constexpr int kSmem = kBarOff + 512 + 1024;
 static_assert(kSmem <= 227 * 1024, "cluster kernel shared memory");
 }  // namespace cl
@@ -1353,7 +1370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const st::Bars sb = st::bars_at(barmem);
   const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + st::kNumBars + ot::kNumBars);
-  volatile long long* ring = reinterpret_cast<volatile long long*>(barmem + st::kNumBars + ot::kNumBars + 1);
+  volatile int4* ring = reinterpret_cast<volatile int4*>(barmem + st::kNumBars + ot::kNumBars + 2);  // 16-byte aligned
   float* part = reinterpret_cast<float*>(smem + cl::kPartOff);
   float* sS = reinterpret_cast<float*>(smem + cl::kScratchOff);
   float* sZ = reinterpret_cast<float*>(smem + cl::kScratchZOff);
