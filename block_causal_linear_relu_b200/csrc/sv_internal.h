@@ -15,6 +15,8 @@ namespace sv {
 //   bytes  8..15  launch sequence number of the one-block kernel (its flags carry it)
 //   bytes 16..19  CTAs of the current one-block launch that have read the sequence number
 //   bytes 24..27  dynamic output-chunk counter of the output kernel (reset by the scan kernel)
+//   bytes 28..35  the one-block kernel's output-chunk counters, one per launch-sequence parity (the
+//                 last CTA to read the sequence number clears the one the next launch uses)
 
 // Tensor maps of one [BH, N, D] bf16 tensor seen as blocks: `main` covers the blocks of length L,
 // `last` the shorter last block when N is not a multiple of L (else it repeats `main`).

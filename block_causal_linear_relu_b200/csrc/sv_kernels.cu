@@ -913,14 +913,17 @@ __global__ void __launch_bounds__(512) scan_kernel(const float* __restrict__ par
 // 4. one launch for one-block problems (bidirectional forward, streaming cache step)
 // ------------------------------------------------------------------------------------------
 // State reduction -> combine -> output in one launch (every CTA resident, one per SM).
-// Each CTA reduces and then outputs the same contiguous tile range; heads are synchronised one by
-// one instead of with grid-wide barriers: a CTA publishes each partial slot it flushes; the CTAs
-// whose range starts inside a head split that head's combine once all its slots are published
-// (reading their share of the incoming cache while they wait, writing the outgoing cache after
-// publishing), and publish their share; a head's output starts once its combine is complete.
-// Flags carry the workspace's launch sequence number (header bytes 8..15, advanced by the last CTA
-// to read it), so nothing needs resetting. The stage memory of the reduction is reused by the output,
-// whose first Q tiles load while the combine runs.
+// Each CTA reduces a contiguous tile range; heads are synchronised one by one instead of with
+// grid-wide barriers: a CTA publishes each partial slot it flushes; the CTAs whose range starts
+// inside a head split that head's combine once all its slots are published (reading their share of
+// the incoming cache while they wait, writing the outgoing cache after publishing), and publish
+// their share; a head's output tiles start once its combine is complete. The output tiles are a
+// static range per CTA plus chunks of the last ~1/8 of the tiles handed out through a counter, as
+// in the output kernel. Flags carry the workspace's launch sequence number (header bytes 8..15,
+// advanced by the last CTA to read it), so nothing needs resetting; that CTA also clears the chunk
+// counter of the next launch (header bytes 28..35, one per parity of the sequence number). The
+// stage memory of the reduction is reused by the output, whose first Q tiles load while the
+// combine runs.
 namespace fu {
 constexpr int kRegion = (st::kRegionBytes > ot::kRegionBytes) ? st::kRegionBytes : ot::kRegionBytes;
 constexpr int kSmem = kRegion + 512 + 1024;
@@ -1128,6 +1131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int4* ring = reinterpret_cast<volatile int4*>(flushed + 2);  // 16-byte aligned
   uint64_t* seqp = reinterpret_cast<uint64_t*>(status + 2);  // header bytes 8..15: launch sequence number
   uint32_t* gstart = status + 4;                             // header bytes 16..19: CTAs that read the tag
+  uint32_t* chunks = status + 7;  // header bytes 28..35: output-chunk counters, one per launch-tag parity
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -1165,6 +1169,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // next launch reads it only after this one has completed.
     if (atom_add_acq_rel_u32(gstart, 1u) == static_cast<uint32_t>(G - 1)) {
       *gstart = 0u;
+      // The chunk counter of the other parity was last used by the previous launch, which has
+      // completed (this one passed griddepcontrol.wait); the next launch uses it, and it claims
+      // chunks only after this launch has completed.
+      chunks[(tag + 1) & 1] = 0u;
       st_release_u64(seqp, tag);
     }
     griddep_launch_dependents();  // the next launch may now set up on SMs as they free up
@@ -1188,7 +1196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // phase 2: the Q stages fill (Q does not depend on the state, and the stages are free once the
   // state MMAs retired) while the CTA takes its share of the combine of its head(s): whole prefix
   // rows, so each cache element belongs to exactly one CTA.
-  const ot::Seq sq{tb, te, 0, 0, nullptr, ring};
+  // The output tiles: a static range of the first T - tdyn tiles, then chunks of the last tdyn
+  // claimed through this launch's counter, so that the CTAs end together: the next launch's CTAs
+  // wait on one another, so every call pays for this launch's slowest CTA.
+  const ot::Seq sq{out_tile_begin(g, geo), out_tile_begin(g + 1, geo), geo.T - geo.tdyn, geo.T,
+                   geo.tdyn > 0 ? chunks + (tag & 1) : nullptr, ring};
   if (warp == kWarpProducer && lane == 0) pre = ot::prefill(smem, ob, mqo, geo, sq, two_atoms);
   float* sS = reinterpret_cast<float*>(smem + fu::kScratchOff);
   float* sZ = reinterpret_cast<float*>(smem + fu::kScratchZOff);
