@@ -100,6 +100,7 @@ def test_fp32_shapes(sv, B, H, N, D, L):
     (2, 1, 300, 8, 77),        # D = 8: a 16-byte row
     (1, 2, 400, 72, 150),      # D = 72 (second atom holds 8 features)
     (1, 1, 260, 120, 260),     # D = 120, bidirectional
+    (2, 40, 500, 16, 500),     # one block per head, 80 heads: the flag-synchronised kernel, D = 16
 ])
 def test_bf16_shapes(sv, B, H, N, D, L):
     st, (q, k, v) = inputs((B, H, N, D), 1, "bf16")
@@ -126,7 +127,7 @@ def test_bf16_many_tiles_per_cta(sv):
 # --------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("B,H,N,D", [(1, 20, 800, 128), (2, 10, 2760, 128), (1, 24, 1000, 112),
                                      (1, 20, 1500, 64), (1, 20, 700, 96), (1, 20, 900, 32),
-                                     (1, 16, 1200, 40)])
+                                     (1, 16, 1200, 40), (1, 20, 600, 24)])
 def test_one_block_few_heads_with_cache(sv, B, H, N, D):
     st, (q, k, v) = inputs((B, H, N, D), 5, "bf16")
     g = np.random.default_rng(7)
