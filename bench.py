@@ -121,14 +121,14 @@ def _blas_threads():
 
 
 def oracle_rate(q, k, v, budget_s: float, max_heads: int | None = None):
-    """Time the fp64 oracle (as it stands) head by head on the stored inputs until budget_s elapse.
-    Returns (tokens*heads per second, heads done, tokens per head, seconds)."""
+    """Time the fp64 oracle (as it stands) head by head on the stored inputs, cycling over the heads,
+    until budget_s elapse (or max_heads heads are done). Returns (tokens*heads per second, heads
+    done, tokens per head, seconds)."""
     import oracle
     from block_causal_linear_relu_b200.inputs import to_f64
 
     done, t0 = 0, time.perf_counter()
-    limit = max_heads if max_heads is not None else H
-    while done < limit:
+    while max_heads is None or done < max_heads:
         h = done % H
         qh, kh, vh = (to_f64(x[:, h:h + 1], "bf16") for x in (q, k, v))
         oracle.block_causal_attn(qh, kh, vh, L, EPS)
@@ -338,8 +338,8 @@ def run_ours(args, rank: int, world: int):
     if world == 1 and not args.no_cpu_baseline:
         rate, nh, ntok, secs = oracle_rate(qs, ks, vs, args.cpu_budget)
         cpu = {"value": rate, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-               "sample": f"fp64 numpy oracle (state form) on {nh} of {H} heads x {ntok} tokens of this "
-                         f"workload, {secs:.1f} s"}
+               "sample": f"fp64 numpy oracle (state form), {nh} heads x {ntok} tokens cycling over this "
+                         f"workload's {H} heads ({nh / H:.1f} passes), {secs:.1f} s"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
