@@ -359,6 +359,10 @@ EXTRA_WORKLOADS = {
     "720p_stream": ("autoregressive cache streaming: 60 blocks of B=1 H=20 N=2760 D=128 through the fp32 cache "
                     "(S [1,20,128,128], z [1,20,128]), one sv_cache_step per block", 1, 20, 2760, 128, 2760,
                     "stream", 60),
+    "720p_denoise": ("autoregressive generation with several denoising steps per block: 12 blocks x 4 steps of "
+                     "B=1 H=20 N=2760 D=128 through the fp32 cache; steps 1-3 of a block attend to it with "
+                     "commit=0, step 4 commits the block's state; fresh q, k, v per step", 1, 20, 2760, 128, 2760,
+                     "denoise", 48),
     "sv2_stack": ("SANA-Video 2.0-shaped stack: 24 bidirectional layers of B=2 H=20 N=10120 D=128, fresh inputs "
                   "per layer, back to back on one stream", 2, 20, 10120, 128, 10120, "fwd", 24),
 }
@@ -383,16 +387,21 @@ def run_extra(args, name):
     outs = [torch.empty_like(x[0]) for x in sets]
     S = torch.zeros(b, h, d, d, device=dev)
     z = torch.zeros(b, h, d, device=dev)
-    op = sv.SV_OP_CACHE_STEP if kind == "stream" else sv.SV_OP_LINATTN_FWD
+    op = sv.SV_OP_LINATTN_FWD if kind == "fwd" else sv.SV_OP_CACHE_STEP
     ws = sv.make_workspace(op, sets[0][0])
     stream = torch.cuda.current_stream()
+    steps_per_block = 4 if kind == "denoise" else 1
+
+    def call(i, st):
+        q, k, v = sets[i]
+        if kind == "fwd":
+            sv.sv_linattn_fwd(q, k, v, o=outs[i], ws=ws, stream=st)
+        else:  # a block's last step commits its state to the cache
+            sv.sv_cache_step(q, k, v, S, z, commit=(i % steps_per_block == steps_per_block - 1), o=outs[i], ws=ws,
+                             stream=st)
 
     def one(i):
-        q, k, v = sets[i]
-        if kind == "stream":
-            sv.sv_cache_step(q, k, v, S, z, commit=True, o=outs[i], ws=ws, stream=stream)
-        else:
-            sv.sv_linattn_fwd(q, k, v, o=outs[i], ws=ws, stream=stream)
+        call(i, stream)
 
     for i in range(min(reps, 3)):
         one(i)
@@ -415,11 +424,7 @@ def run_extra(args, name):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side):
             for i in range(reps):
-                q, k, v = sets[i]
-                if kind == "stream":
-                    sv.sv_cache_step(q, k, v, S, z, commit=True, o=outs[i], ws=ws, stream=side)
-                else:
-                    sv.sv_linattn_fwd(q, k, v, o=outs[i], ws=ws, stream=side)
+                call(i, side)
         graph.replay()
         side.synchronize()
         nrep = max(1, args.steps // reps)

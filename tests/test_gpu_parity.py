@@ -214,6 +214,35 @@ def test_streaming_matches_prefill_and_oracle(sv, dtype):
     assert ws.status() == 0
 
 
+@pytest.mark.parametrize("B,H,N,D", [(1, 20, 600, 128), (1, 4, 300, 64)])
+def test_denoising_steps_per_block(sv, B, H, N, D):
+    # several denoising steps per block, each with fresh q, k, v: steps attend to the cache plus
+    # their own block; only the block's last step commits (20 heads: one cluster per head; 4 heads:
+    # the flag-synchronised kernel)
+    steps, nblocks = 3, 2
+    S = torch.zeros(B, H, D, D, device="cuda")
+    z = torch.zeros(B, H, D, device="cuda")
+    S_ref = np.zeros((B, H, D, D))
+    z_ref = np.zeros((B, H, D))
+    ws = None
+    for c in range(nblocks):
+        for t in range(steps):
+            st, (q, k, v) = inputs((B, H, N, D), 100 + 10 * c + t, "bf16")
+            qd, kd, vd = (dev(x, "bf16") for x in st)
+            if ws is None:
+                ws = sv.make_workspace(sv.SV_OP_CACHE_STEP, qd)
+            commit = t == steps - 1
+            o = sv.sv_cache_step(qd, kd, vd, S, z, commit=commit, eps=EPS, ws=ws)
+            torch.cuda.synchronize()
+            ref, S_new, z_new = oracle.block_causal_attn(q, k, v, N, EPS, S_ref, z_ref)
+            assert oracle.max_rel_err(host(o), ref) < TOL["bf16"]
+            if commit:
+                S_ref, z_ref = S_new, z_new
+            assert oracle.max_rel_err(host(S), S_ref) < TOL_CACHE
+            assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
+    assert ws.status() == 0
+
+
 def test_nonpositive_query_rows_give_exact_zero(sv):
     st, _ = inputs((1, 2, 300, 128), 8, "bf16")
     q = st[0].copy()
