@@ -43,6 +43,8 @@ def lib_path() -> str:
 def load() -> ctypes.CDLL:
     """Load libsvlinattn.so (built in-tree by block_causal_linear_relu_b200.build)."""
     global _lib
+    if _lib is not None:  # loaded: no lock on the per-call path
+        return _lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -92,25 +94,30 @@ def _dt(t: torch.Tensor) -> int:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # plain ints (and None) convert to the c_void_p parameters without a ctypes object per call
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    return stream.cuda_stream
 
 
 def _qkv(*ts):
+    """Checks q, k, v (and o) in one pass; returns their shape [B, H, N, D]."""
     ref = ts[0]
+    shape, dtype, device = ref.shape, ref.dtype, ref.device
+    if not ref.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if len(shape) != 4:
+        raise ValueError("q, k, v, o must share shape [B, H, N, D], dtype and device")
     for t in ts:
-        if not t.is_cuda:
-            raise ValueError("tensors must live on a CUDA device")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous [B, H, N, D]")
-        if t.dim() != 4 or t.shape != ref.shape or t.dtype != ref.dtype or t.device != ref.device:
+        if t is not ref and (t.shape != shape or t.dtype != dtype or t.device != device):
             raise ValueError("q, k, v, o must share shape [B, H, N, D], dtype and device")
-    return ref.shape
+    return shape
 
 
 def workspace_bytes(op: int, B: int, H: int, N: int, D: int, block_len: int, dtype: int, device=None) -> int:
@@ -129,11 +136,12 @@ class Workspace:
         off = (-self.buf.data_ptr()) % 256
         self.view = self.buf[off:off + nbytes]
         self.nbytes = nbytes
-        _check(load().sv_workspace_init(ctypes.c_void_p(self.view.data_ptr()), nbytes, _stream(stream)))
+        self._ptr = self.view.data_ptr()
+        _check(load().sv_workspace_init(self._ptr, nbytes, _stream(stream)))
 
     @property
     def ptr(self):
-        return ctypes.c_void_p(self.view.data_ptr())
+        return self._ptr
 
     def status(self, stream=None) -> int:
         code = ctypes.c_uint32(0)
@@ -161,9 +169,8 @@ def _ws(ws, op, q_like, block_len, stream):
 
 def sv_linattn_fwd(q, k, v, o=None, eps: float = 1e-6, ws: Workspace | None = None, stream=None):
     """Bidirectional ReLU linear attention; returns o."""
-    B, H, N, D = _qkv(q, k, v)
     o = torch.empty_like(q) if o is None else o
-    _qkv(q, o)
+    B, H, N, D = _qkv(q, k, v, o)
     ws = _ws(ws, SV_OP_LINATTN_FWD, q, None, stream)
     _check(load().sv_linattn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, ws.ptr, ws.nbytes,
                                  _stream(stream)))
@@ -173,9 +180,8 @@ def sv_linattn_fwd(q, k, v, o=None, eps: float = 1e-6, ws: Workspace | None = No
 def sv_block_causal_attn(q, k, v, block_len: int, o=None, eps: float = 1e-6, S_in=None, z_in=None, S_out=None,
                          z_out=None, ws: Workspace | None = None, stream=None):
     """Block-causal prefill; returns o (S_out/z_out are written in place when given)."""
-    B, H, N, D = _qkv(q, k, v)
     o = torch.empty_like(q) if o is None else o
-    _qkv(q, o)
+    B, H, N, D = _qkv(q, k, v, o)
     for t in (S_in, z_in, S_out, z_out):
         if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != q.device):
             raise ValueError("S/z must be contiguous float32 tensors on q's device")
@@ -189,9 +195,8 @@ def sv_block_causal_attn(q, k, v, block_len: int, o=None, eps: float = 1e-6, S_i
 def sv_cache_step(q, k, v, S, z, commit: bool = True, o=None, eps: float = 1e-6, ws: Workspace | None = None,
                   stream=None):
     """One streaming block against the fp32 cache (S [B,H,D,D], z [B,H,D]); returns o."""
-    B, H, N, D = _qkv(q, k, v)
     o = torch.empty_like(q) if o is None else o
-    _qkv(q, o)
+    B, H, N, D = _qkv(q, k, v, o)
     if S.dtype != torch.float32 or z.dtype != torch.float32 or tuple(S.shape) != (B, H, D, D) or tuple(z.shape) != (B, H, D):
         raise ValueError("cache must be float32 S [B,H,D,D] and z [B,H,D]")
     ws = _ws(ws, SV_OP_CACHE_STEP, q, None, stream)
@@ -202,9 +207,8 @@ def sv_cache_step(q, k, v, S, z, commit: bool = True, o=None, eps: float = 1e-6,
 
 def sv_cache_step_noalloc(q, k, v, S, z, commit: bool = True, o=None, eps: float = 1e-6, stream=None):
     """sv_cache_step with the library's static scratch instead of a workspace (see the header)."""
-    B, H, N, D = _qkv(q, k, v)
     o = torch.empty_like(q) if o is None else o
-    _qkv(q, o)
+    B, H, N, D = _qkv(q, k, v, o)
     if S.dtype != torch.float32 or z.dtype != torch.float32 or tuple(S.shape) != (B, H, D, D) or tuple(z.shape) != (B, H, D):
         raise ValueError("cache must be float32 S [B,H,D,D] and z [B,H,D]")
     _check(load().sv_cache_step_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, _ptr(S),
