@@ -461,7 +461,7 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
       load_q(smem, b, m, geo, c, s, two_atoms, pol);
     }
   }
-  if (ok) {  // end of the sequence: a plain arrival completes the next stage's qfull with index -1
+  if (ok) {  // end of the sequence: a plain arrival completes the next stage's qfull, its ring entry segment -1
     const int s = k % kStages;
     if (k < pre || mbar_wait(&b.qempty[s], ((k / kStages) & 1) ^ 1, status, 0x1140u | s)) {
       ring_end(sq, k);
