@@ -14,9 +14,11 @@
 //   3. out_bf16_kernel    : per tile, TMA Q -> ReLU(Q) in shared memory -> tcgen05.mma
 //      ReLU(Q) x [P | z]^T into TMEM; the epilogue divides numerator by (denominator + eps),
 //      converts to bf16 and TMA-stores the tile.
-// When every head is a single block (bidirectional layer, streaming step), fused_bf16_kernel runs
-// the three steps in one launch of co-resident CTAs: the state roles, a per-head combine shared by
-// the CTAs that cover the head (synchronised through release/acquire flags), then the output roles.
+// When every head is a single block (bidirectional layer, streaming step), one launch runs the three
+// steps: cluster_bf16_kernel when the heads are few (one thread-block cluster per head, the partial
+// states exchanged through distributed shared memory), otherwise fused_bf16_kernel (co-resident CTAs:
+// the state roles, a per-head combine shared by the CTAs that cover the head, synchronised through
+// release/acquire flags, then the output roles).
 // The fp32 I/O path runs the same three steps with SIMT fp32 kernels.
 #include <cuda_bf16.h>
 
@@ -64,9 +66,10 @@ __device__ __forceinline__ bool use_last_map(const TileCoord& c, const Geom& g) 
 
 // ------------------------------------------------------------------------------------------
 // Pipeline roles. Each persistent kernel runs one CTA per SM with ten warps: warps 0-3 drain the
-// TMEM accumulator (epilogue), warps 4-7 apply ReLU in shared memory, one thread of warp 8 issues
-// TMA copies, one thread of warp 9 issues tcgen05.mma. The roles below are shared by the stand-alone
-// kernels and by the fused single-launch kernel.
+// TMEM accumulator (epilogue), warps 4-7 apply ReLU in shared memory (and, in the output roles with
+// D > 64, drain the second half of the output columns), one thread of warp 8 issues TMA copies, one
+// thread of warp 9 issues tcgen05.mma. The roles below are shared by the stand-alone kernels and by
+// the single-launch kernels.
 // ------------------------------------------------------------------------------------------
 struct Maps4 {
   const CUtensorMap* a_main;
@@ -1228,7 +1231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
 
-  // phase 3: output of the same tiles, each head as soon as its combine is complete
+  // phase 3: the output tiles (static range, then claimed chunks), each once its head's combine is
+  // complete
   if (s_ok) {
     if (warp == kWarpProducer) {
       if (lane == 0) ot::produce(smem, ob, mqo, geo, sq, pre, two_atoms, ptiles, combined, tag, status);
