@@ -5,8 +5,9 @@ Workload (one "step"): the 720p block-causal prefill, B=1, H=20, D=128, 920 toke
 frame (23 x 40), blocks of 3 frames = 2760 tokens, 20 blocks = 55,200 tokens; bf16 q, k, v drawn
 N(0, 1) with numpy's seeded generator (seed = rank), fp32 accumulation, eps = 1e-6, final fp32
 cache written. One step is one call of sv_block_causal_attn: state reduction -> prefix scan ->
-output GEMM, i.e. every step of the hot path. Inputs (565 MB per step) are larger than the 126 MB
-L2, so L2 is not flushed between steps.
+output GEMM, i.e. every step of the hot path. Each step reads q, k and v (848 MB) and writes o
+(283 MB); each kernel streams more than the 126 MB L2 (state: k and v, 565 MB; output: q and o),
+so L2 is not flushed between steps.
 
   python bench.py [--gpus N --steps K --warmup W]        our CUDA path (torchrun for N > 1)
   python bench.py --impl reference [...]                 the fp64 CPU oracle on the host cores
@@ -40,7 +41,7 @@ WORKLOAD = {
                 "x 23x40) D=128, bf16 q/k/v ~ N(0,1), fp32 accumulation, eps=1e-6, final fp32 cache out",
     "B": B, "H": H, "N": N, "D": D, "block_len": L,
     "seed": "rank",
-    "l2": "inputs 565 MB per step > 126 MB L2; not flushed",
+    "l2": "per step q, k, v 848 MB read, o 283 MB written, each kernel streaming > 126 MB L2; not flushed",
 }
 ALG_BYTES_PER_TOKHEAD = 4 * D * 2              # read q, k, v once, write o once (bf16)
 ALG_FLOPS_PER_TOKHEAD = 4 * D * D + 4 * D       # state 2D^2 + z D, numerator 2D^2 + den 2D + div D
