@@ -72,3 +72,36 @@ def test_validation_rejects_before_any_launch(lib):
     su = lib.sv_block_state_update
     assert su(fake, fake, 1, 1, 128, 128, 0, fake, None, fake, 1 << 30, None) == 1
     assert lib.sv_workspace_init(None, 0, None) == 1
+
+
+def test_binding_rejects_bad_tensors_before_the_library():
+    # the binding's single pass of checks: host tensors, wrong rank, mismatched shape or dtype and
+    # non-contiguous tensors raise before any library or CUDA call
+    import torch
+
+    import block_causal_linear_relu_b200 as sv
+    from block_causal_linear_relu_b200 import _native as nat
+
+    q = torch.zeros(1, 2, 64, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA device"):
+        nat._qkv(q, q, q)
+    with pytest.raises(ValueError, match="CUDA device"):
+        sv.sv_linattn_fwd(q, q, q, o=q)
+
+
+def test_cpu_baseline_cycles_over_heads_until_its_budget():
+    # the CPU oracle baseline keeps cycling over the workload's heads until its time budget is
+    # spent (more heads than the workload holds), and max_heads caps it
+    import bench
+    from block_causal_linear_relu_b200.inputs import draw_qkv
+
+    saved = (bench.H, bench.N, bench.L)
+    try:
+        bench.H, bench.N, bench.L = 2, 96, 32
+        q, k, v = draw_qkv((1, 2, 96, 16), 0, "bf16")
+        rate, heads, ntok, secs = bench.oracle_rate(q, k, v, 0.2)
+        assert heads > bench.H and ntok == 96 and secs >= 0.2 and rate > 0
+        _, heads1, _, _ = bench.oracle_rate(q, k, v, 0.0, max_heads=1)
+        assert heads1 == 1
+    finally:
+        bench.H, bench.N, bench.L = saved
