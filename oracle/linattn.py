@@ -33,8 +33,9 @@ O_i = phi(q_i)^T P_blk(i) / (phi(q_i)^T zP_blk(i) + eps).
 Pins (tests/test_oracle_pins.py): two independent brute forces of the explicit masked N x N
 matrix (numpy here, plain C in bruteforce.c), the token recurrence of causal linear attention
 (Katharopoulos et al. 2020) for L = 1, closed forms (constant v, non-positive q row, one-hot
-state), and invariants (streaming == prefill, constant cache bytes, permutation within a block).
-Every function below is pinned; none is "parity unpinned".
+state), small cases worked by hand from the definition (tests/golden, one of them with an
+incoming cache and eps > 0), and invariants (streaming == prefill, constant cache bytes,
+permutation within a block). Every function below is pinned; none is "parity unpinned".
 """
 
 from __future__ import annotations

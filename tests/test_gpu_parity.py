@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import golden
 import oracle
 from block_causal_linear_relu_b200.inputs import draw_qkv, to_f64
 
@@ -241,6 +242,33 @@ def test_denoising_steps_per_block(sv, B, H, N, D):
             assert oracle.max_rel_err(host(S), S_ref) < TOL_CACHE
             assert oracle.max_rel_err(host(z), z_ref) < TOL_CACHE
     assert ws.status() == 0
+
+
+@pytest.mark.parametrize("name", golden.FIXTURES)
+def test_hand_worked_fixtures_fp32(sv, name):
+    # the hand-worked cases of tests/golden through the fp32 path; the API takes D value features,
+    # so v (and the cache) carry the fixture's E columns followed by zero columns (outputs 0 there)
+    g = golden.load(name)
+    D, E = g["D"], g["E"]
+    N = g["q"].shape[2]
+    v = np.zeros((1, 1, N, D))
+    v[..., :E] = g["v"]
+    qd, kd, vd = (dev(x.astype(np.float32), "f32") for x in (g["q"], g["k"], v))
+    for blen, key in ((g["block_len"], "o_block_causal"), (N, "o_bidirectional")):
+        kw = {}
+        if "S_in" in g:
+            S0 = np.zeros((1, 1, D, D), np.float32)
+            S0[..., :E] = g["S_in"]
+            kw = dict(S_in=torch.from_numpy(S0).cuda(), z_in=torch.from_numpy(g["z_in"].astype(np.float32)).cuda(),
+                      S_out=torch.zeros(1, 1, D, D, device="cuda"), z_out=torch.zeros(1, 1, D, device="cuda"))
+        o = sv.sv_block_causal_attn(qd, kd, vd, blen, eps=g["eps"], **kw)
+        torch.cuda.synchronize()
+        got = host(o)
+        assert np.allclose(got[..., :E], g[key], rtol=1e-5, atol=1e-6), (got[..., :E], g[key])
+        assert np.all(got[..., E:] == 0.0)
+        if kw and key == "o_block_causal":
+            assert np.allclose(host(kw["S_out"])[..., :E], g["S_out"], rtol=1e-6, atol=1e-6)
+            assert np.allclose(host(kw["z_out"]), g["z_out"], rtol=1e-6, atol=1e-6)
 
 
 def test_nonpositive_query_rows_give_exact_zero(sv):

@@ -52,3 +52,25 @@ def test_planted_eps_in_numerator_is_caught_by_zero_row():
     q[0, 0, 5] = -1.0  # a non-positive query row must give exactly zero
     out = _mutant("eps_in_numerator", q, k, v, 8, 1e-3)
     assert np.any(out[0, 0, 5] != 0.0)
+
+
+@pytest.mark.parametrize("kind", ["cache_ignored", "cache_twice", "cache_z_dropped"])
+def test_planted_cache_mistake_is_caught_by_hand_worked_fixture(kind):
+    # the incoming cache's handling, against the hand-worked fixture with a cache (tests/golden)
+    import golden
+
+    g = golden.load("hand_worked_cache_d1_n3.txt")
+    S, z = L.block_states(g["k"], g["v"], g["block_len"])
+    S_in, z_in = g["S_in"], g["z_in"]
+    if kind == "cache_ignored":
+        S_in, z_in = None, None
+    elif kind == "cache_twice":
+        S_in, z_in = 2 * S_in, 2 * z_in
+    elif kind == "cache_z_dropped":
+        z_in = None
+    P, zP = L.prefix_states(S, z, S_in, z_in)
+    got = L.apply_states(g["q"], P, zP, g["block_len"], g["eps"])
+    assert not np.allclose(got, g["o_block_causal"], rtol=1e-6, atol=1e-9)
+    P0, zP0 = L.prefix_states(S, z, g["S_in"], g["z_in"])
+    assert np.allclose(L.apply_states(g["q"], P0, zP0, g["block_len"], g["eps"]), g["o_block_causal"], rtol=1e-15,
+                       atol=1e-15)

@@ -14,6 +14,7 @@ sign in the feature map) fails at least one of them:
 import numpy as np
 import pytest
 
+import golden
 import oracle
 from oracle.bruteforce import bruteforce_c
 from block_causal_linear_relu_b200.inputs import draw_qkv, to_f64
@@ -79,19 +80,22 @@ def test_block_len_at_least_n_is_bidirectional():
     assert np.array_equal(a, b) and np.array_equal(a, c)
 
 
-def test_hand_worked_example():
-    # D=2, N=4, L=2, eps=0, worked by hand from the definition.
-    # phi(q) = [[1,0],[0,1],[1,1],[0,2]], phi(k) = [[2,0],[0,1],[1,0],[1,1]], v = [1,2,3,4].
-    # block-causal: token0 sees j<2: A=[2,0] -> 2/2=1; token1: A=[0,1] -> 2/1=2;
-    #   token2 sees all: A=[2,1,1,2] -> (2+2+3+8)/6 = 2.5; token3: A=[0,2,0,2] -> (4+8)/4 = 3.
-    # bidirectional: token0: A=[2,0,1,1] -> (2+3+4)/4 = 2.25; token1: A=[0,1,0,1] -> (2+4)/2 = 3.
-    q = np.array([[1, 0], [0, 1], [1, 1], [-1, 2]], float)[None, None]
-    k = np.array([[2, 0], [0, 1], [1, -1], [1, 1]], float)[None, None]
-    v = np.array([[1], [2], [3], [4]], float)[None, None]
-    bc = oracle.block_causal_attn(q, k, v, 2, 0.0)[0][0, 0, :, 0]
-    bi = oracle.linattn_fwd(q, k, v, 0.0)[0, 0, :, 0]
-    assert np.allclose(bc, [1.0, 2.0, 2.5, 3.0], rtol=0, atol=1e-15)
-    assert np.allclose(bi, [2.25, 3.0, 2.5, 3.0], rtol=0, atol=1e-15)
+@pytest.mark.parametrize("name", golden.FIXTURES)
+def test_hand_worked_fixtures(name):
+    # tests/golden: small cases worked by hand from the definition (the derivations are in the files)
+    g = golden.load(name)
+    S_in, z_in = g.get("S_in"), g.get("z_in")
+    o, S_out, z_out = oracle.block_causal_attn(g["q"], g["k"], g["v"], g["block_len"], g["eps"], S_in, z_in)
+    assert np.allclose(o, g["o_block_causal"], rtol=1e-15, atol=1e-15)
+    if S_in is not None:
+        assert np.allclose(S_out, g["S_out"], rtol=0, atol=1e-15)
+        assert np.allclose(z_out, g["z_out"], rtol=0, atol=1e-15)
+    n = g["q"].shape[2]
+    ob = oracle.block_causal_attn(g["q"], g["k"], g["v"], n, g["eps"], S_in, z_in)[0]
+    assert np.allclose(ob, g["o_bidirectional"], rtol=1e-15, atol=1e-15)
+    if S_in is None:
+        assert np.allclose(oracle.linattn_fwd(g["q"], g["k"], g["v"], g["eps"]), g["o_bidirectional"], rtol=1e-15,
+                           atol=1e-15)
 
 
 def test_uniform_attention_is_running_mean():
