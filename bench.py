@@ -164,7 +164,8 @@ def run_reference(args, rank: int, world: int):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": WORKLOAD,
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu_model": _cpu_model(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -338,9 +339,14 @@ def run_ours(args, rank: int, world: int):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         rate, nh, ntok, secs = oracle_rate(qs, ks, vs, args.cpu_budget)
-        cpu = {"value": rate, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+        cpu = {"value": rate, "unit": UNIT, "cores": _blas_threads(), "cpu_model": _cpu_model(), "kind": "oracle",
                "sample": f"fp64 numpy oracle (state form), {nh} heads x {ntok} tokens cycling over this "
                          f"workload's {H} heads ({nh / H:.1f} passes), {secs:.1f} s"}
+    extras = None
+    if world == 1 and not args.no_extras:
+        extras = {}
+        for name, passes in EXTRA_PASSES.items():
+            extras[name] = time_workload(name, passes, dev.index)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -348,6 +354,7 @@ def run_ours(args, rank: int, world: int):
         "roofline": roofline, "step_roofline": step_roof,
         "kernels_ms": kernels, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
         "gpu_launches": 3 * args.steps, "impl": "ours",
+        "other_configs": extras,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -369,17 +376,30 @@ EXTRA_WORKLOADS = {
 }
 
 
-def run_extra(args, name):
-    """Timing of the other configurations (one JSON line; not the default bench line). Inputs come
-    from torch's seeded CUDA generator (seed 0), distinct per layer / per block."""
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def time_workload(name, passes: int, dev_index: int = 0):
+    """Device time of one of the other configurations, as a dict for the bench line. Every call of a
+    pass gets distinct inputs (torch's seeded CUDA generator, seed 0), so L2 never holds a call's
+    inputs from an earlier call. Eager: CUDA events around each call issued from Python through the
+    binding. Graph: one pass of the same calls captured in a CUDA graph and replayed (how a
+    generation loop issues them), device time per call."""
     import torch
 
     import block_causal_linear_relu_b200 as sv
 
     desc, b, h, n, d, blen, kind, reps = EXTRA_WORKLOADS[name]
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    sv.load()
+    dev = torch.device("cuda", dev_index)
     hbm_gbs, _, _, _ = peaks()
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
@@ -401,25 +421,20 @@ def run_extra(args, name):
             sv.sv_cache_step(q, k, v, S, z, commit=(i % steps_per_block == steps_per_block - 1), o=outs[i], ws=ws,
                              stream=st)
 
-    def one(i):
-        call(i, stream)
-
     for i in range(min(reps, 3)):
-        one(i)
+        call(i, stream)
     torch.cuda.synchronize()
     per = []
-    for _ in range(max(1, args.steps // reps)):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
-        evs[0].record(stream)
-        for i in range(reps):
-            one(i)
-            evs[i + 1].record(stream)
-        torch.cuda.synchronize()
-        per += [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
-    # the same sequence of calls captured once in a CUDA graph and replayed: per-call device time
-    # without the host's per-call launch work (how a generation loop would issue the calls)
-    graph_ms = None
-    side = torch.cuda.Stream()
+    with ClockSampler(dev.index) as clk_e:
+        for _ in range(passes):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+            evs[0].record(stream)
+            for i in range(reps):
+                call(i, stream)
+                evs[i + 1].record(stream)
+            torch.cuda.synchronize()
+            per += [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
+    side = torch.cuda.Stream(device=dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
         graph = torch.cuda.CUDAGraph()
@@ -428,30 +443,53 @@ def run_extra(args, name):
                 call(i, side)
         graph.replay()
         side.synchronize()
-        nrep = max(1, args.steps // reps)
         ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ga.record(side)
-        for _ in range(nrep):
-            graph.replay()
-        gb.record(side)
-        side.synchronize()
-        graph_ms = ga.elapsed_time(gb) / (nrep * reps)
+        with ClockSampler(dev.index) as clk_g:
+            ga.record(side)
+            for _ in range(passes):
+                graph.replay()
+            gb.record(side)
+            side.synchronize()
+        graph_ms = ga.elapsed_time(gb) / (passes * reps)
     del graph
     torch.cuda.synchronize()
     if ws.status() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     per_ms = np.array(per)
     tokheads = b * h * n
-    ms = float(per_ms.mean())
-    step_bytes = tokheads * 4 * d * 2
-    line = {"metric": METRIC, "value": tokheads / (ms / 1e3), "unit": UNIT, "n_gpus": 1, "workload": name,
-            "config": {"workload": desc}, "calls_timed": len(per), "ms_per_call_mean": ms,
-            "ms_per_call_median": float(np.median(per_ms)), "ms_per_call_p90": float(np.percentile(per_ms, 90)),
-            "hbm_gbs_alg": step_bytes / (ms / 1e3) / 1e9, "hbm_frac": step_bytes / (ms / 1e3) / 1e9 / hbm_gbs,
-            "graph": {"ms_per_call": graph_ms, "value": tokheads / (graph_ms / 1e3),
-                      "hbm_frac": step_bytes / (graph_ms / 1e3) / 1e9 / hbm_gbs,
-                      "timing": "the same calls captured in one CUDA graph, replayed; CUDA events"},
-            "dtype": "bf16", "data": "synthetic (torch CUDA generator, seed 0)", "impl": "ours"}
+    call_bytes = tokheads * 4 * d * 2
+    t_roof_ms = call_bytes / (hbm_gbs * 1e9) * 1e3
+    gl = 3 if blen < n else 1
+    return {
+        "workload": desc, "B": b, "H": h, "N": n, "D": d, "block_len": blen, "calls_per_pass": reps,
+        "passes": passes, "kernels_per_call": gl, "gpu_launches": gl * reps * passes * 2,
+        "alg_bytes_per_call": call_bytes, "t_roof_ms": t_roof_ms,
+        "graph": {"ms_per_call": graph_ms, "value": tokheads / (graph_ms / 1e3), "hbm_frac": t_roof_ms / graph_ms,
+                  "clocks": clk_g.summary()},
+        "eager": {"ms_per_call_mean": float(per_ms.mean()), "ms_per_call_median": float(np.median(per_ms)),
+                  "ms_per_call_p90": float(np.percentile(per_ms, 90)), "value": tokheads / (per_ms.mean() / 1e3),
+                  "hbm_frac": t_roof_ms / float(per_ms.mean()), "clocks": clk_e.summary()},
+        "unit": UNIT, "data": "synthetic (torch CUDA generator, seed 0), distinct inputs per call",
+        "timing": "CUDA events; eager = per call from Python, graph = one pass captured and replayed",
+    }
+
+
+# passes of each other configuration timed inside the default bench run (each pass: every call of
+# the workload once, with distinct inputs)
+EXTRA_PASSES = {"480p_bidir": 200, "720p_stream": 5, "sv2_stack": 8, "720p_denoise": 4}
+
+
+def run_extra(args, name):
+    """One configuration alone, as an informational JSON line (not the bench line)."""
+    import torch
+
+    import block_causal_linear_relu_b200 as sv
+
+    torch.cuda.set_device(0)
+    sv.load()
+    r = time_workload(name, max(1, args.steps // EXTRA_WORKLOADS[name][-1]))
+    line = {"metric": METRIC, "value": r["graph"]["value"], "unit": UNIT, "n_gpus": 1, "workload": name,
+            "impl": "ours", "dtype": "bf16", **r}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -466,6 +504,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="leave the other configurations (480p, streaming, 2.0 stack, denoising) out of the line")
     ap.add_argument("--workload", choices=["720p_prefill"] + sorted(EXTRA_WORKLOADS), default="720p_prefill",
                     help="the bench line is 720p_prefill; the others print an informational timing line")
     ap.add_argument("--heads", type=int, default=None,

@@ -22,6 +22,7 @@ from ._native import (  # noqa: F401
     sv_block_state_update,
     sv_cache_step,
     sv_cache_step_noalloc,
+    sv_cache_step_noalloc_status,
     sv_linattn_fwd,
     sv_profile_events,
     sv_selftest_wait_timeout,

@@ -24,9 +24,10 @@ SV_OP_LINATTN_FWD, SV_OP_BLOCK_STATE_UPDATE, SV_OP_BLOCK_CAUSAL_ATTN, SV_OP_CACH
 
 #: every symbol include/svlinattn.h declares
 EXPORTS = (
-    "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_linattn_fwd",
+    "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_workspace_set_mirror", "sv_linattn_fwd",
     "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_cache_step_noalloc",
-    "sv_profile_events", "sv_last_error", "sv_selftest_wait_timeout", "sv_version",
+    "sv_cache_step_noalloc_status", "sv_profile_events", "sv_last_error", "sv_selftest_wait_timeout",
+    "sv_version",
 )
 
 
@@ -58,6 +59,8 @@ def load() -> ctypes.CDLL:
         lib.sv_workspace_init.restype = i
         lib.sv_device_status.argtypes = [vp, vp, u32p]
         lib.sv_device_status.restype = i
+        lib.sv_workspace_set_mirror.argtypes = [vp, sz, vp, vp]
+        lib.sv_workspace_set_mirror.restype = i
         lib.sv_linattn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
         lib.sv_linattn_fwd.restype = i
         lib.sv_block_state_update.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, sz, vp]
@@ -68,6 +71,8 @@ def load() -> ctypes.CDLL:
         lib.sv_cache_step.restype = i
         lib.sv_cache_step_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, vp, vp, i, vp]
         lib.sv_cache_step_noalloc.restype = i
+        lib.sv_cache_step_noalloc_status.argtypes = [vp, u32p]
+        lib.sv_cache_step_noalloc_status.restype = i
         lib.sv_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
         lib.sv_profile_events.restype = i
         lib.sv_last_error.argtypes = []
@@ -129,7 +134,13 @@ def workspace_bytes(op: int, B: int, H: int, N: int, D: int, block_len: int, dty
 
 
 class Workspace:
-    """Caller-owned device scratch: a 256-byte aligned view into a torch uint8 buffer."""
+    """Caller-owned device scratch: a 256-byte aligned view into a torch uint8 buffer.
+
+    A page-locked host word is registered as the workspace's status mirror: a kernel whose bounded
+    wait expires writes its status code there as well, so every later call of this binding on the
+    workspace raises SvError(SV_ERR_TIMEOUT) before it launches anything (``check``), without a
+    synchronisation per call. ``status`` synchronises, reads and clears the device word.
+    """
 
     def __init__(self, nbytes: int, device, stream=None):
         self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
@@ -137,18 +148,33 @@ class Workspace:
         self.view = self.buf[off:off + nbytes]
         self.nbytes = nbytes
         self._ptr = self.view.data_ptr()
-        _check(load().sv_workspace_init(self._ptr, nbytes, _stream(stream)))
+        self._mirror = torch.zeros(1, dtype=torch.int32).pin_memory()
+        self._mirror_np = self._mirror.numpy()
+        lib = load()
+        with torch.cuda.device(self.buf.device):
+            _check(lib.sv_workspace_init(self._ptr, nbytes, _stream(stream)))
+            _check(lib.sv_workspace_set_mirror(self._ptr, nbytes, self._mirror.data_ptr(), _stream(stream)))
 
     @property
     def ptr(self):
         return self._ptr
 
     def status(self, stream=None) -> int:
+        """Synchronise, return the device status word (0 = no timeout) and clear it (and the mirror)."""
         code = ctypes.c_uint32(0)
         st = load().sv_device_status(self.ptr, _stream(stream), ctypes.byref(code))
         if st not in (SV_OK, SV_ERR_TIMEOUT):
             _check(st)
+        self._mirror_np[0] = 0
         return int(code.value)
+
+    def check(self, stream=None):
+        """Raise SvError(SV_ERR_TIMEOUT) if a kernel has reported a timeout on this workspace since the
+        last check (reads the host mirror: no synchronisation unless a timeout was reported)."""
+        if self._mirror_np[0] != 0:
+            code = self.status(stream)
+            raise SvError(SV_ERR_TIMEOUT, f"a kernel's bounded wait expired on this workspace "
+                                          f"(status word 0x{code:08x}); its output was not written")
 
 
 def sv_selftest_wait_timeout(ws: Workspace, stream=None):
@@ -163,8 +189,20 @@ def make_workspace(op: int, q_like: torch.Tensor, block_len: int | None = None, 
     return Workspace(n, q_like.device, stream)
 
 
+_default_ws = {}
+
+
 def _ws(ws, op, q_like, block_len, stream):
-    return ws if ws is not None else make_workspace(op, q_like, block_len, stream)
+    """The caller's workspace, else one kept per (device, stream, op, sizes), so that calls without
+    an explicit workspace reuse it (calls on one stream are ordered) and see its reported timeouts."""
+    if ws is None:
+        B, H, N, D = q_like.shape
+        key = (q_like.device.index, _stream(stream), op, B, H, N, D, block_len, q_like.dtype)
+        ws = _default_ws.get(key)
+        if ws is None:
+            ws = _default_ws[key] = make_workspace(op, q_like, block_len, stream)
+    ws.check(stream)
+    return ws
 
 
 def sv_linattn_fwd(q, k, v, o=None, eps: float = 1e-6, ws: Workspace | None = None, stream=None):
@@ -214,6 +252,16 @@ def sv_cache_step_noalloc(q, k, v, S, z, commit: bool = True, o=None, eps: float
     _check(load().sv_cache_step_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, _dt(q), eps, _ptr(S),
                                         _ptr(z), 1 if commit else 0, _stream(stream)))
     return o
+
+
+def sv_cache_step_noalloc_status(stream=None) -> int:
+    """Synchronise and return (then clear) the status word of sv_cache_step_noalloc's static scratch
+    on the current device (0 = no timeout)."""
+    code = ctypes.c_uint32(0)
+    st = load().sv_cache_step_noalloc_status(_stream(stream), ctypes.byref(code))
+    if st not in (SV_OK, SV_ERR_TIMEOUT):
+        _check(st)
+    return int(code.value)
 
 
 def sv_profile_events(events):

@@ -310,6 +310,29 @@ sv_status sv_workspace_init(void* ws, size_t ws_bytes, sv_stream_t stream) {
   return SV_OK;
 }
 
+sv_status sv_workspace_set_mirror(void* ws, size_t ws_bytes, uint32_t* host_word, sv_stream_t stream) {
+  if (ws == nullptr || ws_bytes < static_cast<size_t>(sv::kHeaderBytes) || !aligned(ws, 256))
+    return fail(SV_ERR_INVALID_ARG, "workspace is NULL, not 256-byte aligned or smaller than %d bytes",
+                sv::kHeaderBytes);
+  void* dptr = nullptr;
+  if (host_word != nullptr) {
+    if (!aligned(host_word, 4)) return fail(SV_ERR_INVALID_ARG, "host_word is not 4-byte aligned");
+    const cudaError_t e = cudaHostGetDevicePointer(&dptr, host_word, 0);
+    if (e != cudaSuccess || dptr == nullptr) {
+      (void)cudaGetLastError();
+      return fail(SV_ERR_INVALID_ARG, "host_word is not page-locked host memory the device can write (%s)",
+                  cudaGetErrorName(e));
+    }
+  }
+  // a pageable source is staged by the runtime before cudaMemcpyAsync returns
+  const uint64_t addr = reinterpret_cast<uint64_t>(dptr);
+  cudaError_t e = cudaMemcpyAsync(static_cast<uint8_t*>(ws) + 4 * sv::kMirrorWord, &addr, sizeof(addr),
+                                  cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "writing the mirror address into the workspace header");
+  return SV_OK;
+}
+
 sv_status sv_device_status(void* ws, sv_stream_t stream, uint32_t* code) {
   if (ws == nullptr) return fail(SV_ERR_INVALID_ARG, "workspace is NULL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

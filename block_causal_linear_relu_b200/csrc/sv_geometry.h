@@ -33,6 +33,7 @@ constexpr int kOutChunk = 4;      // tiles per dynamically handed-out output chu
 constexpr int kHeaderBytes = 256;                            // status word(s) at the workspace start
 
 constexpr uint32_t kDevTimeout = 0x80000000u;                // status bit: a bounded wait expired
+constexpr int kMirrorWord = 10;  // header bytes 40..47 (32-bit word 10): device address of a host-mapped status copy
 constexpr uint64_t kWaitLimitNs = 2000000000ull;             // 2 s per wait
 
 struct Geom {

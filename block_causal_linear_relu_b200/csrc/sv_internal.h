@@ -17,6 +17,8 @@ namespace sv {
 //   bytes 24..27  dynamic output-chunk counter of the output kernel (reset by the scan kernel)
 //   bytes 28..35  the one-block kernel's output-chunk counters, one per launch-sequence parity (the
 //                 last CTA to read the sequence number clears the one the next launch uses)
+//   bytes 40..47  device address of a host-mapped copy of the status word, or 0 (set by
+//                 sv_workspace_set_mirror; a kernel that raises the status word also stores it there)
 
 // Tensor maps of one [BH, N, D] bf16 tensor seen as blocks: `main` covers the blocks of length L,
 // `last` the shorter last block when N is not a multiple of L (else it repeats `main`).

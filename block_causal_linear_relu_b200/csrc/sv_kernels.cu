@@ -121,7 +121,7 @@ __device__ bool wait_flags(const uint64_t* flags, int i0, int i1, uint64_t tag, 
     if (ready < n) {
       if (*reinterpret_cast<volatile uint32_t*>(status) != 0u) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, kDevTimeout | where);
+        raise_status(status, kDevTimeout | where);
         return false;
       }
       __nanosleep(32);

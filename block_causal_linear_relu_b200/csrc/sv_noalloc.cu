@@ -13,10 +13,15 @@
 //    this array until the process exits, whether or not the entry point is used;
 //  - a call whose workspace need (sv_workspace_bytes(SV_OP_CACHE_STEP, ...)) exceeds the array is
 //    refused with SV_ERR_INVALID_ARG before anything is launched;
-//  - all calls on a device share the one array, which keeps the previous call's contents: calls
-//    that may overlap on the GPU (different streams without ordering) race on it;
-//  - the first call on each device looks up the array's device address with that device current;
-//    make that first call before any stream capture begins.
+//  - all calls on a device share the one array, which keeps the previous call's contents (the
+//    status word, the one-launch kernel's sequence number and flags): calls that may overlap on the
+//    GPU (different streams without ordering) race on it;
+//  - the first call on each device (or of sv_cache_step_noalloc_status) looks up the array's device
+//    address with that device current and keeps it for the life of the process; make that first
+//    call before any stream capture begins. After cudaDeviceReset the kept address is stale: the
+//    entry point is not supported across a device reset.
+//  - a bounded wait that expires raises the array's status word, which stays raised (later calls
+//    then give up their waits at once) until sv_cache_step_noalloc_status reads and clears it.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -37,6 +42,30 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
+// Device address of the scratch on the current device, looked up once per device.
+sv_status scratch_address(void** out, const char* who) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    char msg[160];
+    snprintf(msg, sizeof(msg), "%s: no usable current device", who);
+    return sv::set_last_error(SV_ERR_CUDA, msg);
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      char msg[200];
+      snprintf(msg, sizeof(msg), "%s: cudaGetSymbolAddress of the static scratch failed (%s)", who,
+               cudaGetErrorName(e));
+      return sv::set_last_error(SV_ERR_CUDA, msg);
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SV_OK;
+}
+
 }  // namespace
 
 extern "C" sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N,
@@ -52,26 +81,19 @@ extern "C" sv_status sv_cache_step_noalloc(const void* q, const void* k, const v
              need, kNoAllocScratchBytes);
     return sv::set_last_error(SV_ERR_INVALID_ARG, msg);
   }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return sv::set_last_error(SV_ERR_CUDA, "sv_cache_step_noalloc: no usable current device");
   void* ws = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-      void* p = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess || p == nullptr)
-        return sv::set_last_error(SV_ERR_CUDA,
-                                  "sv_cache_step_noalloc: cudaGetSymbolAddress of the static scratch failed");
-      g_scratch_addr[dev] = p;
-    }
-    ws = g_scratch_addr[dev];
-  }
-  // the status word must start at zero; the launch sequence number and the flags behind it keep
-  // their values from call to call (the array starts zeroed when the library loads), and the rest is
-  // fully rewritten by each call
-  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return sv::set_last_error(SV_ERR_CUDA, "sv_cache_step_noalloc: clearing the scratch header failed");
+  const sv_status s = scratch_address(&ws, "sv_cache_step_noalloc");
+  if (s != SV_OK) return s;
+  // Nothing is written here: the array starts zeroed when the library loads, the status word is
+  // cleared only by sv_cache_step_noalloc_status, the launch sequence number and the flags behind it
+  // keep their values from call to call, and the rest is rewritten by each call. sv_cache_step
+  // checks every argument before it launches anything.
   return sv_cache_step(q, k, v, o, B, H, N, D, dt, eps, S, z, commit, ws, kNoAllocScratchBytes, stream);
+}
+
+extern "C" sv_status sv_cache_step_noalloc_status(sv_stream_t stream, uint32_t* code) {
+  void* ws = nullptr;
+  const sv_status s = scratch_address(&ws, "sv_cache_step_noalloc_status");
+  if (s != SV_OK) return s;
+  return sv_device_status(ws, stream, code);
 }

@@ -59,6 +59,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Raises the workspace status word (bytes 0..3) to `code` and, when the caller registered one
+// (header bytes 40..47, see sv_workspace_set_mirror), stores the code into a host-mapped word as
+// well, so that the host sees the failure without synchronising. Failure path only.
+static __device__ __noinline__ void raise_status(uint32_t* status, uint32_t code) {
+  atomicOr(status, code);
+  uint32_t* mirror = *reinterpret_cast<uint32_t* const volatile*>(status + kMirrorWord);
+  if (mirror != nullptr) {
+    *reinterpret_cast<volatile uint32_t*>(mirror) = code;
+    __threadfence_system();
+  }
+}
+
 // Slow path of a bounded wait: polls until the phase with `parity` completes, another thread of the
 // grid has raised the status word, or kWaitLimitNs elapse (then it raises SV_DEV_TIMEOUT | where).
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status,
@@ -69,7 +81,7 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     if ((it & 63u) == 0u) {
       if (*reinterpret_cast<volatile uint32_t*>(status) != 0u) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, kDevTimeout | where);
+        raise_status(status, kDevTimeout | where);
         return false;
       }
     }

@@ -27,7 +27,10 @@
  *    Calls that share one workspace must be ordered on the GPU (same stream, or synchronised).
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *    Pointers stay owned by the caller; the library allocates nothing and keeps no state
- *    between calls other than per-device kernel attributes.
+ *    between calls other than per-device kernel attributes, with one exception: the library
+ *    holds a static 16 MiB device array on every device that loads it, the scratch of
+ *    sv_cache_step_noalloc, whose contents (status word, launch sequence number, flags) persist
+ *    from one call of that entry point to the next.
  *  - Supported sizes: B, H, N >= 1; SV_BF16: D a multiple of 8 in [8, 128] (a row must be a whole
  *    number of 16-byte units); SV_F32: 1 <= D <= 128. eps must be finite and >= 0.
  *  - Errors: every argument is checked on the host BEFORE anything is launched; a bad argument
@@ -83,8 +86,21 @@ size_t sv_workspace_bytes(sv_op op, int B, int H, int N, int D, int block_len, s
 sv_status sv_workspace_init(void* ws, size_t ws_bytes, sv_stream_t stream);
 
 /* Synchronise `stream`, read the workspace's status word and clear it. SV_OK if no kernel
- * raised it; SV_ERR_TIMEOUT if a bounded wait expired (the word is then in *code, if given). */
+ * raised it; SV_ERR_TIMEOUT if a bounded wait expired (the word is then in *code, if given).
+ * Until it is cleared, a raised word makes every later call on this workspace give up its waits at
+ * once (its output is then not written): a timeout is sticky, like a CUDA error. */
 sv_status sv_device_status(void* ws, sv_stream_t stream, uint32_t* code);
+
+/* Register a host word that the kernels also write when they raise the workspace's status word, so
+ * that a caller learns of a device-side timeout without synchronising (for instance by checking the
+ * word before each call, as the Python binding does). host_word must be page-locked host memory
+ * that the device can write (cudaHostAlloc / cudaMallocHost; with unified addressing every such
+ * allocation is mapped), 4-byte aligned, and must outlive the workspace's use; NULL removes the
+ * registration. The caller clears host_word itself (sv_device_status clears only the device word).
+ * Synchronises `stream`. Call after sv_workspace_init, which clears the registration. Returns
+ * SV_ERR_INVALID_ARG for a bad workspace or a host_word the device cannot write. Not a step of the
+ * method: failure reporting of this library. */
+sv_status sv_workspace_set_mirror(void* ws, size_t ws_bytes, uint32_t* host_word, sv_stream_t stream);
 
 /* Bidirectional full-sequence linear attention (the Linear DiT layer: every token attends to
  * every token of its (b, h) sequence; SANA-Video abstract, design (1) "Linear DiT"):
@@ -94,13 +110,19 @@ sv_status sv_linattn_fwd(const void* q, const void* k, const void* v, void* o, i
 
 /* Add a block's state to the cache in place (talk, block KV cache passage: the state is updated
  * additively, the current block's contribution added to the previous cache):
- *     S += phi(K)^T V,  z += sum_j phi(k_j)  over the N tokens of k, v ([B, H, N, D]). */
+ *     S += phi(K)^T V,  z += sum_j phi(k_j)  over the N tokens of k, v ([B, H, N, D]).
+ * Unlike a plain cache update this call takes a workspace (sv_workspace_bytes with
+ * SV_OP_BLOCK_STATE_UPDATE): the reduction is spread over every streaming multiprocessor, and their
+ * partial states are combined there before S and z are written. */
 sv_status sv_block_state_update(const void* k, const void* v, int B, int H, int N, int D, sv_dtype dt, float* S,
                                 float* z, void* ws, size_t ws_bytes, sv_stream_t stream);
 
 /* Block-causal prefill over a whole sequence cut into blocks of block_len tokens (the last block
- * may be shorter). Token i of block c = floor(i / block_len) attends to every token of blocks
- * 0..c plus the incoming cache:
+ * may be shorter), as in the talk's block-causal walkthrough: block 1's state is cached, block 2's
+ * contribution is added to that cache, and so on, so that every block sees the summed state of all
+ * blocks before it; within its own block a token sees every token (the block is diffused as a
+ * whole: talk, hybrid AR + diffusion passage). Token i of block c = floor(i / block_len) attends to
+ * every token of blocks 0..c plus the incoming cache:
  *     P_c = S_in + sum_{c' <= c} S_c',  zP_c = z_in + sum_{c' <= c} z_c',
  *     o_i = phi(q_i) P_c / (phi(q_i) . zP_c + eps).
  * S_in/z_in (nullable: zero cache) is the cache before the sequence; S_out/z_out (nullable: not
@@ -130,11 +152,18 @@ sv_status sv_cache_step(const void* q, const void* k, const void* v, void* o, in
  * SV_OP_CACHE_STEP: about 66 KB per (batch, head) pair plus 66 KB per streaming multiprocessor,
  * so the 720p streaming block [1, 20, 2760, 128] needs about 12 MB and B * H above ~100 does not
  * fit) is refused with SV_ERR_INVALID_ARG before any launch. All calls on a device share the
- * array: calls that may overlap on the GPU race. The first call on a device looks up the array's
- * device address; make it before any stream capture. Device-side wait timeouts are not reported through this entry
- * point (use sv_cache_step with a workspace and sv_device_status for that). */
+ * array, which keeps the previous call's contents: calls that may overlap on the GPU race. The
+ * first call on a device looks up the array's device address and keeps it for the life of the
+ * process; make it before any stream capture, and do not use this entry point across a
+ * cudaDeviceReset. A device-side wait timeout raises the array's status word, which stays raised
+ * (later calls then give up at once) until sv_cache_step_noalloc_status reads and clears it. */
 sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
                                 sv_dtype dt, float eps, float* S, float* z, int commit, sv_stream_t stream);
+
+/* sv_device_status for the static scratch of sv_cache_step_noalloc on the current device:
+ * synchronises `stream`, reads the array's status word and clears it (SV_OK, or SV_ERR_TIMEOUT with
+ * the word in *code if given). Allocates nothing. */
+sv_status sv_cache_step_noalloc_status(sv_stream_t stream, uint32_t* code);
 
 /* Optional timing hook for benchmarks. With events != NULL (n == 4 cudaEvent_t handles owned by
  * the caller), the calling thread's following forward calls (sv_linattn_fwd, sv_block_causal_attn,

@@ -56,3 +56,33 @@ def test_selftest_refuses_bad_workspace(sv):
     assert lib.sv_selftest_wait_timeout(ctypes.c_void_p(ws.view.data_ptr() + 8), 4088, None) == invalid
     assert lib.sv_selftest_wait_timeout(ws.ptr, 64, None) == invalid
     assert ws.status() == 0                     # nothing was launched
+
+
+def test_binding_raises_on_the_next_call_after_a_timeout(sv):
+    # a kernel that gives up a bounded wait also writes its code into the workspace's host-mapped
+    # mirror word; the binding reads that word before each call and raises instead of launching on a
+    # workspace whose last call did not complete (no per-call synchronisation)
+    st = draw_qkv((1, 2, 300, 64), 12, "bf16")
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda() for x in st)
+    ws = sv.make_workspace(sv.SV_OP_LINATTN_FWD, q)
+    sv.sv_selftest_wait_timeout(ws)
+    torch.cuda.synchronize()                    # the waiters give up after about 2 s
+    with pytest.raises(sv.SvError) as err:
+        sv.sv_linattn_fwd(q, k, v, eps=1e-6, ws=ws)
+    assert err.value.status == 4                # SV_ERR_TIMEOUT
+    # the check read and cleared the word: the next call runs, and correctly
+    o = sv.sv_linattn_fwd(q, k, v, eps=1e-6, ws=ws)
+    torch.cuda.synchronize()
+    want = oracle.linattn_fwd(*(to_f64(x, "bf16") for x in st), 1e-6)
+    assert oracle.max_rel_err(o.float().cpu().numpy().astype(np.float64), want) < 2e-2
+    ws.check()                                  # nothing reported since
+
+
+def test_mirror_needs_host_memory_the_device_can_write(sv):
+    import ctypes
+    lib = sv.load()
+    ws = sv.Workspace(4096, torch.device("cuda:0"))
+    dev_word = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert lib.sv_workspace_set_mirror(ws.ptr, ws.nbytes, ctypes.c_void_p(dev_word.data_ptr()), None) == 1
+    assert b"page-locked" in lib.sv_last_error()
+    assert lib.sv_workspace_set_mirror(ws.ptr, ws.nbytes, None, None) == 0   # removing it is allowed
