@@ -17,3 +17,5 @@ from .linattn import (  # noqa: F401
     prefix_states,
     rows_from_states,
 )
+from .projection import out_projection, qkv_projection  # noqa: F401,E402
+from .temporal_conv import centred_conv, temporal_conv_block_causal, temporal_conv_step  # noqa: F401,E402

@@ -35,3 +35,16 @@ def load(name: str) -> dict:
 
 
 FIXTURES = ["hand_worked_d2_n4.txt", "hand_worked_cache_d1_n3.txt"]
+
+
+def load_values(name: str) -> dict:
+    """Parse any fixture into {key: float64 array} ('#' lines are comments)."""
+    vals = {}
+    with open(os.path.join(HERE, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = np.array([float(x) for x in rest])
+    return vals
