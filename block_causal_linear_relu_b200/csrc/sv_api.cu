@@ -90,8 +90,47 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Encoded maps of this thread's recent calls: an encoding depends only on the key below, so a hit
+// is exactly the map the driver would encode again (a streaming loop reuses its buffers call after
+// call, and each encode costs about a microsecond of host time).
+struct MapKey {
+  const void* base;
+  uint64_t rows, nblk;
+  int D, L, N, BH;
+  uint32_t box_rows;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && nblk == o.nblk && D == o.D && L == o.L && N == o.N && BH == o.BH &&
+           box_rows == o.box_rows;
+  }
+};
+constexpr int kMapCache = 32;
+thread_local MapKey g_map_keys[kMapCache];
+thread_local CUtensorMap g_maps[kMapCache];
+thread_local int g_map_count = 0, g_map_next = 0;
+
+sv_status encode_map_uncached(CUtensorMap* m, const void* base, uint64_t rows, uint64_t nblk, const Geom& g,
+                              uint32_t box_rows);
+
 sv_status encode_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t nblk, const Geom& g,
                      uint32_t box_rows) {
+  const MapKey key{base, rows, nblk, g.D, g.L, g.N, g.BH, box_rows};
+  for (int i = 0; i < g_map_count; ++i)
+    if (g_map_keys[i] == key) {
+      *m = g_maps[i];
+      return SV_OK;
+    }
+  const sv_status s = encode_map_uncached(m, base, rows, nblk, g, box_rows);
+  if (s != SV_OK) return s;
+  const int i = g_map_next;
+  g_map_next = (g_map_next + 1) % kMapCache;
+  if (g_map_count < kMapCache) ++g_map_count;
+  g_map_keys[i] = key;
+  g_maps[i] = *m;
+  return SV_OK;
+}
+
+sv_status encode_map_uncached(CUtensorMap* m, const void* base, uint64_t rows, uint64_t nblk, const Geom& g,
+                              uint32_t box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return fail(SV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const uint64_t D = static_cast<uint64_t>(g.D);
@@ -228,22 +267,36 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
   void* pre = wsb + lay.ptiles;
   cudaError_t e;
   if (dt == SV_BF16) {
+    // one block per head and few heads: one thread-block cluster per head (a single launch)
+    const int C = g.nblk == 1 ? sv::cluster_size(g, di.sm_count) : 0;
+    if (C > 0) {
+      sv::ClusterMaps cm;
+      SV_TRY(encode_map(&cm.k, k, g.N, 1, g, sv::kTile));
+      SV_TRY(encode_map(&cm.v, v, g.N, 1, g, sv::kTile));
+      SV_TRY(encode_map(&cm.q, q, g.N, 1, g, sv::kTile));
+      SV_TRY(encode_map(&cm.o, o, g.N, 1, g, 32));
+      SV_TRY(encode_map(&cm.k16, k, g.N, 1, g, 16));
+      SV_TRY(encode_map(&cm.v16, v, g.N, 1, g, 16));
+      SV_TRY(encode_map(&cm.q16, q, g.N, 1, g, 16));
+      SV_TRY(encode_map(&cm.o16, o, g.N, 1, g, 16));
+      prof_mark(0, stream);
+      e = sv::launch_cluster_bf16(cm, g, C, partials, S_in, z_in, S_out, z_out, eps, status, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "cluster kernel launch");
+      prof_mark(1, stream);
+      prof_mark(2, stream);
+      prof_mark(3, stream);
+      return SV_OK;
+    }
     sv::BlockMaps mq, mk, mv, mo;
     SV_TRY(make_block_maps(mk, k, g, sv::kTile));
     SV_TRY(make_block_maps(mv, v, g, sv::kTile));
     SV_TRY(make_block_maps(mq, q, g, sv::kTile));
     SV_TRY(make_block_maps(mo, o, g, 32));
-    if (g.nblk == 1) {  // one block: a single launch, one cluster per head when the heads are few
+    if (g.nblk == 1) {  // one block per head, many heads: a single launch of co-resident CTAs
       prof_mark(0, stream);
-      const int C = sv::cluster_size(g, di.sm_count);
-      if (C > 0) {
-        e = sv::launch_cluster_bf16(mk, mv, mq, mo, g, C, S_in, z_in, S_out, z_out, eps, status, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "cluster kernel launch");
-      } else {
-        e = sv::launch_fused_bf16(mk, mv, mq, mo, g, partials, segcta, flags, pre, S_in, z_in, S_out, z_out, eps,
-                                  status, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
-      }
+      e = sv::launch_fused_bf16(mk, mv, mq, mo, g, partials, segcta, flags, pre, S_in, z_in, S_out, z_out, eps,
+                                status, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
       prof_mark(1, stream);
       prof_mark(2, stream);
       prof_mark(3, stream);

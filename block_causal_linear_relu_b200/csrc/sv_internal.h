@@ -37,12 +37,18 @@ cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const Bloc
                               const Geom& g, float* partials, int2* segcta, uint64_t* flags, void* ptiles,
                               const float* S_in, const float* z_in, float* S_out, float* z_out, float eps,
                               uint32_t* status, cudaStream_t st);
-// bf16, whole sequence in one block, few heads: one thread-block cluster of C CTAs per head.
+// bf16, whole sequence in one block, few heads: one thread-block cluster of C CTAs per head, whose
+// ranks split the head's rows in 16-row units. Maps of the one-block [BH, N, D] tensors: k, v, q
+// with 128-row boxes, o with 32-row store boxes, and the same four with 16-row boxes. The head's
+// summed state is reduced in `accum` (fp32 [BH][129][128] in the workspace).
 // cluster_size returns the C to use for this geometry (0: use launch_fused_bf16 instead).
+struct ClusterMaps {
+  CUtensorMap k, v, q, o, k16, v16, q16, o16;
+};
 int cluster_size(const Geom& g, int sm_count);
-cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
-                                const Geom& g, int C, const float* S_in, const float* z_in, float* S_out,
-                                float* z_out, float eps, uint32_t* status, cudaStream_t st);
+cudaError_t launch_cluster_bf16(const ClusterMaps& m, const Geom& g, int C, float* accum, const float* S_in,
+                                const float* z_in, float* S_out, float* z_out, float eps, uint32_t* status,
+                                cudaStream_t st);
 // fp32 path
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
                              uint32_t* status, cudaStream_t st);

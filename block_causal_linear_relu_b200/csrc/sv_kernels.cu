@@ -973,55 +973,6 @@ __device__ void combine_load_cache(const Geom& geo, const float* S_in, const flo
     for (int d = tid; d < D; d += nthr) sZ[d] = __ldcg(z_in + static_cast<size_t>(bh) * D + d);
 }
 
-// The same two steps for a share whose bounds are multiples of 4 (float4 along e when the cache is
-// 16-byte aligned; the API only promises 4-byte alignment, so otherwise element by element).
-__device__ void combine_load_cache_q(const Geom& geo, const float* S_in, const float* z_in, int bh, int r0, int r1,
-                                     float* sS, float* sZ, int tid, int nthr) {
-  const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1), nq = ns / 4;
-  if (S_in != nullptr) {
-    const float* src = S_in + static_cast<size_t>(bh) * D * D + r0;
-    if ((reinterpret_cast<uintptr_t>(S_in) & 15u) == 0u) {
-      for (int i = tid; i < D * nq; i += nthr) {
-        const int d = i / nq, j = (i - d * nq) * 4;
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + static_cast<size_t>(d) * D + j));
-        sS[(j + 0) * ld + d] = v.x;
-        sS[(j + 1) * ld + d] = v.y;
-        sS[(j + 2) * ld + d] = v.z;
-        sS[(j + 3) * ld + d] = v.w;
-      }
-    } else {
-      for (int i = tid; i < D * ns; i += nthr) {
-        const int d = i / ns, j = i - d * ns;
-        sS[j * ld + d] = __ldcg(src + static_cast<size_t>(d) * D + j);
-      }
-    }
-  }
-  if (z_in != nullptr && r0 <= kZRow && kZRow < r1)
-    for (int d = tid; d < D; d += nthr) sZ[d] = __ldcg(z_in + static_cast<size_t>(bh) * D + d);
-}
-
-__device__ void combine_store_cache_q(const Geom& geo, float* S_out, float* z_out, int bh, int r0, int r1,
-                                      const float* sS, const float* sZ, int tid, int nthr) {
-  const int D = geo.D, ld = D + 1, ns = cache_rows(geo, r0, r1), nq = ns / 4;
-  if (S_out != nullptr) {
-    float* dst = S_out + static_cast<size_t>(bh) * D * D + r0;
-    if ((reinterpret_cast<uintptr_t>(S_out) & 15u) == 0u) {
-      for (int i = tid; i < D * nq; i += nthr) {
-        const int d = i / nq, j = (i - d * nq) * 4;
-        *reinterpret_cast<float4*>(dst + static_cast<size_t>(d) * D + j) =
-            make_float4(sS[(j + 0) * ld + d], sS[(j + 1) * ld + d], sS[(j + 2) * ld + d], sS[(j + 3) * ld + d]);
-      }
-    } else {
-      for (int i = tid; i < D * ns; i += nthr) {
-        const int d = i / ns, j = i - d * ns;
-        dst[static_cast<size_t>(d) * D + j] = sS[j * ld + d];
-      }
-    }
-  }
-  if (z_out != nullptr && r0 <= kZRow && kZRow < r1)
-    for (int d = tid; d < D; d += nthr) z_out[static_cast<size_t>(bh) * D + d] = sZ[d];
-}
-
 // Step 2 (once the head's partial slots exist): each row = cache + the slots of CTAs g0..g1 in
 // ascending order, written as the bf16 B operand of the output GEMM; the sums replace the cache
 // values in sS / sZ for step 3. Each thread takes two (row, quad) items per pass and keeps up to 8
@@ -1253,140 +1204,441 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------------------
 // 5. one block per head with one thread-block cluster per head (few heads, e.g. a streaming step)
 // ------------------------------------------------------------------------------------------
-// Cluster h (C CTAs) owns head h; rank r reduces tiles [r*tph/C, (r+1)*tph/C) of the head into
-// TMEM exactly as the state roles do, then drains its partial state into its own shared memory.
-// After a cluster barrier each rank sums its share of prefix rows over the C partials, read in rank
-// order through distributed shared memory, adds the incoming cache, and writes the bf16 rows into
-// the prefix tile of every rank of the cluster. After a second cluster barrier every rank holds
-// the whole prefix tile and runs the output roles on its tiles; the outgoing cache is written from
-// the fp32 sums. No global round trip and no flag sits between the reduction and the output.
-// Every thread reaches both cluster barriers on every path (the roles only leave their loops on
-// a failed bounded wait), and no shared memory of another rank is touched after the second one.
+// Cluster h (C CTAs) owns head h. The head's rows are split between the ranks in units of 16 rows
+// (rank r: units [r*U/C, (r+1)*U/C) of the U = ceil(N/16) units), at most 512 rows (4 tiles) per
+// rank, so the busiest rank holds ~N/C rows instead of a whole number of 128-row tiles. A range
+// that ends inside a tile is loaded with 16-row boxes (a 128-row box would read the next rank's
+// rows); the state MMAs of a tile cover only its 16-row steps.
+//   phase 1: rank r reduces its rows into TMEM (the state roles, one segment); meanwhile its
+//            epilogue warps zero its share of the head's fp32 accumulator [129][128] in the
+//            workspace and fetch its share of the incoming cache; after the last state MMA the
+//            producer loads every Q tile of the rank (all of them fit: the stages are free), and
+//            the ReLU warps apply the feature map to each as it lands.
+//   exchange: the epilogue warps drain TMEM into shared memory as [e][d] rows (adding the rank's
+//            share of the incoming cache), and one thread adds them to the head's accumulator
+//            with TMA bulk reductions (cp.reduce.async.bulk .add.f32, in L2), half by half while
+//            the drain goes on. A cluster barrier; then every rank reads the summed state (the
+//            inclusive prefix P, fp32) back, writes it as its bf16 B tile and keeps its share of
+//            rows for the outgoing cache.
+//   phase 3: the output MMAs run back to back over the resident Q tiles; the epilogue stores each
+//            tile's output through the tile's own Q slot (its MMA has read it by then).
+// Two cluster barriers: B1 (accumulator zeroed; split arrive/wait, so nobody waits for it in
+// practice) and B2 (every rank's reduction complete). Both are taken by every thread on every path
+// (bounded mbarrier waits only make roles skip work), without .aligned so a warp's lanes may reach
+// them at different points. The sums in L2 are in arrival order, so the fp32 state (and hence
+// the output) is not bitwise reproducible from call to call on this path; its error stays the
+// fp32 summation error.
 namespace cl {
 constexpr int kMinCluster = 4;
 constexpr int kMaxCluster = 8;
-constexpr int kPartOff = ot::kBOff + kPTileBytes;                // partial [129][128] fp32 (row e, column d)
+constexpr int kUnit = 16;                            // rows per unit of the split between ranks
+constexpr int kMaxTiles = 4;                         // resident Q tiles: at most 512 rows per rank
+constexpr int kQSlot = 2 * kAtomBytes;               // one Q tile (32 KB), later its output staging
+constexpr int kPartOff = kMaxTiles * kQSlot;         // fp32 partial [129][128], later the bf16 B tile
 constexpr int kPartBytes = kPartRows * kDPad * 4;
-static_assert(kPartOff + kPartBytes <= fu::kRegion, "partial state overflows the stage region");
-static_assert(kPartOff >= ot::kBOff + kPTileBytes && kPartOff % 1024 == 0, "partial overlaps the prefix tile");
-static_assert(kPartOff + 2 * 4 * ot::kOWarpBytes <= fu::kRegion, "double-buffered output staging overflows");
+constexpr int kRegion = st::kRegionBytes;
+// The partial overlaps the last K/V stage and the ones tile: both are dead once the state MMAs
+// retired, which the drain waits for.
+static_assert(kPartOff + kPartBytes <= kRegion && kPartOff + kPTileBytes <= kRegion, "partial overflows the region");
+static_assert(kPartOff % 1024 == 0, "B tile alignment");
 constexpr int kShareRowsMax = (kPTileRows + kMinCluster - 1) / kMinCluster;
-constexpr int kScratchOff = fu::kRegion;                          // incoming-cache share, transposed
-constexpr int kScratchZOff = kScratchOff + kShareRowsMax * (kDPad + 1) * 4;
+constexpr int kScratchOff = kRegion;                 // cache share [row][128] fp32 (S_in, then P)
+constexpr int kScratchZOff = kScratchOff + kShareRowsMax * kDPad * 4;
 constexpr int kBarOff = (kScratchZOff + kDPad * 4 + 127) / 128 * 128;
+constexpr int kNumBars = st::kNumBars + 2 * kMaxTiles + 5;
 constexpr int kSmem = kBarOff + 512 + 1024;
+static_assert(kNumBars * 8 + 8 <= 512, "barrier area");
 static_assert(kSmem <= 227 * 1024, "cluster kernel shared memory");
-}  // namespace cl
 
-// Epilogue warps 0-3: the single accumulator of this rank (TMEM lanes = key feature d) into the
-// partial [e][d] in shared memory; row kZRow holds z.
-__device__ void cl_drain_partial(const st::Bars& b, uint32_t tmem, int warp, int lane, float* part,
-                                 uint32_t* status) {
+struct Bars3 {            // phase 3
+  uint64_t* qfull;        // [4] Q tile j landed
+  uint64_t* qrelu;        // [4] ReLU(Q tile j) written back (4 ReLU warps)
+  uint64_t* accf;         // [2] output accumulator holds a tile
+  uint64_t* acce;         // [2] output accumulator drained
+  uint64_t* done;
+};
+__device__ __forceinline__ Bars3 bars3_at(uint64_t* p) {
+  return Bars3{p, p + kMaxTiles, p + 2 * kMaxTiles, p + 2 * kMaxTiles + 2, p + 2 * kMaxTiles + 4};
+}
+
+// Tiles of one rank: tile j starts at row tok0(j) of the head and holds rows(j) rows.
+struct Range {
+  int row0, row1, n, N;
+  __device__ __forceinline__ int tok0(int j) const { return row0 + j * kTile; }
+  __device__ __forceinline__ int rows(int j) const {
+    const int r = row1 - tok0(j);
+    return r < kTile ? r : kTile;
+  }
+  // A tile whose range ends before the head does is loaded with 16-row boxes; one that reaches the
+  // head's end uses whole boxes, clipped (and zero-filled) by the tensor map.
+  __device__ __forceinline__ bool boxed16(int j) const { return rows(j) < kTile && tok0(j) + kTile < N; }
+};
+
+struct Maps {
+  const CUtensorMap* k;    // 128-row boxes
+  const CUtensorMap* v;
+  const CUtensorMap* q;
+  const CUtensorMap* o;    // 32-row store boxes
+  const CUtensorMap* k16;  // 16-row boxes
+  const CUtensorMap* v16;
+  const CUtensorMap* q16;
+  const CUtensorMap* o16;
+};
+
+// non-aligned cluster barrier halves: each thread arrives and waits at its own point
+__device__ __forceinline__ void arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
+__device__ __forceinline__ void wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
+// Loads rows(j) rows of one [BH, N, D] tensor at (tok0, bh) into `dst` (128-row tile layout, one or
+// two 16 KB atoms); returns the bytes the barrier must expect.
+__device__ __forceinline__ uint32_t load_rows(uint8_t* dst, const CUtensorMap* m128, const CUtensorMap* m16,
+                                              uint64_t* bar, const Range& rg, int j, int bh, bool two_atoms,
+                                              uint64_t pol) {
+  const int tok0 = rg.tok0(j);
+  const int na = two_atoms ? 2 : 1;
+  if (!rg.boxed16(j)) {
+    for (int a = 0; a < na; ++a) tma_load_4d(dst + a * kAtomBytes, m128, bar, 64 * a, tok0, 0, bh, pol);
+    return static_cast<uint32_t>(na * kAtomBytes);
+  }
+  const int nb = rg.rows(j) / kUnit;
+  for (int u = 0; u < nb; ++u)
+    for (int a = 0; a < na; ++a)
+      tma_load_4d(dst + a * kAtomBytes + u * (kUnit * 128), m16, bar, 64 * a, tok0 + u * kUnit, 0, bh, pol);
+  return static_cast<uint32_t>(nb * na * kUnit * 128);
+}
+
+// Producer, phase 1: the rank's K and V tiles through the three stages; then, once every state
+// MMA has retired (the stages are free), every Q tile of the rank into its own slot.
+__device__ void produce(uint8_t* smem, const st::Bars& b, const Bars3& b3, const Maps& m, const Range& rg, int bh,
+                        bool two_atoms, uint32_t* status) {
+  const uint64_t pol = policy_evict_first();
+  int j = 0;
+  for (; j < rg.n; ++j) {
+    const int s = j % st::kStages;
+    if (!mbar_wait(&b.empty[s], ((j / st::kStages) & 1) ^ 1, status, 0x3100u | s)) return;
+    uint8_t* stg = smem + s * st::kStageBytes;
+    // both expect_tx before either copy, so the phase cannot complete early
+    const int nb = rg.boxed16(j) ? rg.rows(j) / kUnit : 0;
+    const uint32_t per = nb ? static_cast<uint32_t>(nb * kUnit * 128) : static_cast<uint32_t>(kAtomBytes);
+    mbar_expect_tx(&b.full[s], (two_atoms ? 4u : 2u) * per);
+    load_rows(stg, m.k, m.k16, &b.full[s], rg, j, bh, two_atoms, pol);
+    load_rows(stg + st::kKBytes, m.v, m.v16, &b.full[s], rg, j, bh, two_atoms, pol);
+  }
+  for (int i = (rg.n > st::kStages ? rg.n - st::kStages : 0); i < rg.n; ++i)
+    if (!mbar_wait(&b.empty[i % st::kStages], (i / st::kStages) & 1, status, 0x3180u)) return;
+  for (int i = 0; i < rg.n; ++i) {
+    const int nb = rg.boxed16(i) ? rg.rows(i) / kUnit : 0;
+    const uint32_t per = nb ? static_cast<uint32_t>(nb * kUnit * 128) : static_cast<uint32_t>(kAtomBytes);
+    mbar_expect_tx(&b3.qfull[i], (two_atoms ? 2u : 1u) * per);
+    load_rows(smem + i * kQSlot, m.q, m.q16, &b3.qfull[i], rg, i, bh, two_atoms, pol);
+  }
+}
+
+// MMA issuer, phase 1: ReLU(K)^T [V | 1] over the rank's rows into accumulator 0; only the 16-row
+// steps that hold rows of the range are issued.
+__device__ void mma_state(uint8_t* smem, const st::Bars& b, const Range& rg, uint32_t tmem, uint32_t* status) {
+  constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, true, true);
+  constexpr uint32_t kIdescZ = idesc_bf16_f32(128, 16, true, true);
+  const uint64_t od = sdesc_sw128(smem_u32(smem + st::kOnesOff), kAtomBytes, 1024);
+  for (int j = 0; j < rg.n; ++j) {
+    const int s = j % st::kStages;
+    const uint32_t ph = (j / st::kStages) & 1;
+    if (!mbar_wait(&b.full[s], ph, status, 0x3310u | s)) return;
+    if (!mbar_wait(&b.relu[s], ph, status, 0x3320u | s)) return;
+    tc_fence_after();
+    const uint32_t kb = smem_u32(smem + s * st::kStageBytes);
+    const uint32_t vb = kb + st::kKBytes;
+    const int steps = (rg.rows(j) + kUnit - 1) / kUnit;
+    for (int kk = 0; kk < steps; ++kk) {
+      const uint64_t ad = sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024);
+      const uint64_t bd = sdesc_sw128(vb + kk * 2048, kAtomBytes, 1024);
+      const uint32_t acc = (j == 0 && kk == 0) ? 0u : 1u;
+      mma_bf16(tmem, ad, bd, kIdescS, acc);
+      mma_bf16(tmem + 128, ad, od, kIdescZ, acc);
+    }
+    mma_commit(&b.empty[s]);
+  }
+  mma_commit(&b.accf[0]);
+}
+
+__device__ __forceinline__ void st_shared_f32(uint32_t saddr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(saddr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Rows of the rank's share [r0, r1) that are rows of S (e < D): the incoming and outgoing cache go
+// through sS as [row - r0][128] fp32 (features d >= D zero), z through sZ[128].
+__device__ __forceinline__ int share_rows(const Geom& geo, int r0, int r1) {
+  const int e_hi = r1 < geo.D ? r1 : geo.D;
+  return e_hi > r0 ? e_hi - r0 : 0;
+}
+__device__ __forceinline__ bool share_has_z(int r0, int r1) { return r0 <= kZRow && kZRow < r1; }
+
+// Warps 0-3, phase 1: the share of the incoming cache into sS / sZ (transposed: sS[e - r0][d] =
+// S_in[d][e]), loads batched ahead of the stores. The rows reach the accumulator as one more bulk
+// reduction, so the drain itself only stores.
+__device__ void load_cache_share(const Geom& geo, const float* __restrict__ S_in, const float* __restrict__ z_in,
+                                 int bh, int r0, int r1, float* __restrict__ sS, float* __restrict__ sZ, int tid) {
+  const int D = geo.D, ns = share_rows(geo, r0, r1);
+  if (S_in != nullptr && ns > 0) {
+    for (int i = tid; i < ns * kDPad; i += 128) sS[i] = 0.f;  // features d >= D stay zero
+    __syncwarp();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // items (d, e): consecutive threads take consecutive e of one key row d (coalesced reads)
+    const float* src = S_in + static_cast<size_t>(bh) * D * D + r0;
+    const int items = D * ns;
+    for (int i0 = tid; i0 < items; i0 += 8 * 128) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 128;
+        const int d = i / ns, j = i - d * ns;
+        v[u] = i < items ? __ldcg(src + static_cast<size_t>(d) * D + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 128;
+        const int d = i / ns, j = i - d * ns;
+        if (i < items) sS[j * kDPad + d] = v[u];
+      }
+    }
+  }
+  if (z_in != nullptr && share_has_z(r0, r1))
+    sZ[tid] = tid < D ? __ldcg(z_in + static_cast<size_t>(bh) * D + tid) : 0.f;
+}
+
+// After the read-back (warp 8, overlapping the output): the share of the outgoing cache from sS /
+// sZ. S_out[d][r0 + j] = sS[j][d]: float4 stores along j where the cache is 16-byte aligned (row
+// starts then are too: D and r0 are multiples of 4), gathers batched ahead of the stores.
+__device__ void store_cache_share(const Geom& geo, float* __restrict__ S_out, float* __restrict__ z_out, int bh,
+                                  int r0, int r1, const float* __restrict__ sS, const float* __restrict__ sZ, int tid,
+                                  int nthr) {
+  const int D = geo.D, ns = share_rows(geo, r0, r1);
+  if (S_out != nullptr && ns > 0) {
+    float* dst = S_out + static_cast<size_t>(bh) * D * D + r0;
+    if ((reinterpret_cast<uintptr_t>(S_out) & 15u) == 0u) {
+      const int nq = ns / 4, items = D * nq;  // (d, quad of j)
+      for (int i0 = tid; i0 < items; i0 += 4 * nthr) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * nthr;
+          const int d = i / nq, j = (i - d * nq) * 4;
+          if (i < items)
+            v[u] = make_float4(sS[j * kDPad + d], sS[(j + 1) * kDPad + d], sS[(j + 2) * kDPad + d],
+                               sS[(j + 3) * kDPad + d]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * nthr;
+          const int d = i / nq, j = (i - d * nq) * 4;
+          if (i < items) *reinterpret_cast<float4*>(dst + static_cast<size_t>(d) * D + j) = v[u];
+        }
+      }
+    } else {
+      for (int i = tid; i < D * ns; i += nthr) {
+        const int d = i / ns, j = i - d * ns;
+        dst[static_cast<size_t>(d) * D + j] = sS[j * kDPad + d];
+      }
+    }
+  }
+  if (z_out != nullptr && share_has_z(r0, r1))
+    for (int d = tid; d < D; d += nthr) z_out[static_cast<size_t>(bh) * D + d] = sZ[d];
+}
+
+// Epilogue warps 0-3: the rank's share of the incoming cache goes to the head's accumulator first
+// (bulk reductions of sS / sZ, issued once B1 has published the zeroing); then accumulator 0 (lane =
+// key feature d) is drained into the partial [e][d] in shared memory, and thread 0 adds each
+// drained half to the accumulator with a bulk reduction. Every thread of the four warps passes both
+// named barriers whatever happened before.
+__device__ void drain_reduce(const st::Bars& b, const Geom& geo, uint32_t tmem, int warp, int lane, float* part,
+                             float* acc, bool has_S, bool has_z, int r0, int r1, const float* sS, const float* sZ,
+                             uint32_t* status) {
   const int d = warp * 32 + lane;
-  const bool ok = mbar_wait(&b.accf[0], 0, status, 0x3400u);
-  if (!warp_all(ok)) return;
-  tc_fence_after();
+  const bool ok = warp_all(mbar_wait(&b.accf[0], 0, status, 0x3400u));
+  wait_acquire();  // B1: every rank has zeroed its share of the accumulator
+  if (threadIdx.x == 0) {
+    asm volatile("fence.proxy.async.global;" ::: "memory");  // the zeroing B1 acquired -> async proxy
+    const int ns = share_rows(geo, r0, r1);
+    if (has_S && ns > 0) bulk_reduce_add_f32(acc + r0 * kDPad, sS, static_cast<uint32_t>(ns * kDPad * 4));
+    if (has_z && share_has_z(r0, r1)) bulk_reduce_add_f32(acc + kZRow * kDPad, sZ, kDPad * 4);
+    bulk_commit();
+  }
+  if (ok) tc_fence_after();
   const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint32_t ps = smem_u32(part) + static_cast<uint32_t>(d * 4);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    uint32_t rr[2][32];
-    uint32_t zr = 0;
-    tmem_ld_x32(ta + h * 64, rr[0]);
-    tmem_ld_x32(ta + h * 64 + 32, rr[1]);
-    if (h == 1) tmem_ld_x1(ta + 128, zr);
-    tmem_wait_ld();
+    if (ok) {
+      uint32_t rr[2][32];
+      uint32_t zr = 0;
+      tmem_ld_x32(ta + h * 64, rr[0]);
+      tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+      if (h == 1) tmem_ld_x1(ta + 128, zr);
+      tmem_wait_ld();
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc)
+      for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) part[(h * 64 + cc * 32 + jj) * kDPad + d] = __uint_as_float(rr[cc][jj]);
-    if (h == 1) part[kZRow * kDPad + d] = __uint_as_float(zr);
+        for (int jj = 0; jj < 32; ++jj)
+          st_shared_f32(ps + static_cast<uint32_t>((h * 64 + cc * 32 + jj) * kDPad * 4), __uint_as_float(rr[cc][jj]));
+      if (h == 1) st_shared_f32(ps + static_cast<uint32_t>(kZRow * kDPad * 4), __uint_as_float(zr));
+    }
+    fence_proxy_async_smem();  // these generic writes -> the bulk reduction (async proxy)
+    named_sync(1, 128);
+    if (threadIdx.x == 0) {
+      const int e0 = h * 64, e1 = h == 0 ? 64 : kPartRows;
+      bulk_reduce_add_f32(acc + e0 * kDPad, part + e0 * kDPad, static_cast<uint32_t>((e1 - e0) * kDPad * 4));
+      bulk_commit();
+    }
+  }
+  if (threadIdx.x == 0) {
+    bulk_wait_all();  // the reductions are complete in global memory
+    asm volatile("fence.proxy.async.global;" ::: "memory");  // ... and ordered before the B2 release
   }
   tc_fence_before();
 }
 
-// This rank's share of the head's prefix rows: sum of the C partials (rank order) + cache, bf16 rows
-// written into every rank's prefix tile; the fp32 sums stay in sS / sZ for the outgoing cache.
-__device__ void cl_combine(const Geom& geo, uint32_t part_s, uint32_t ptile_s, int C, int me, bool has_S,
-                           bool has_z, int r0, int r1, float* sS, float* sZ, int tid, int nthr) {
-  const int D = geo.D, ld = D + 1;
-  // two (row, quad) items per thread and pass, the C partial values of both in flight at once
-  for (int base = r0 * 32 + tid; base < r1 * 32; base += 2 * nthr) {
-    float4 p[2][cl::kMaxCluster];
+// Read-back by the 192 threads of warps 0-3, 8 and 9 (index gt): the summed state P (fp32 [129][128]
+// in L2) into the bf16 B tile (rows 129..143 zero), and the rank's share of rows into sS / sZ for
+// the outgoing cache. Twelve (row, 8-feature) items per thread; the loads have no condition (rows
+// past z read row 128 and are zeroed afterwards) so that all 24 are in flight at once.
+__device__ void read_back(const Geom& geo, const float* acc, uint8_t* btile, int r0, int r1, float* __restrict__ sS,
+                          float* __restrict__ sZ, int gt) {
+  constexpr int kGroup = 192, kBatch = 12;
+  static_assert(kGroup * kBatch == kPTileRows * 16, "one batch covers the B tile");
+  const int ns_hi = r0 + share_rows(geo, r0, r1);
+  float4 v[kBatch][2];
 #pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const int it = base + x * nthr;
-      const int e = it >> 5, d0 = (it & 31) * 4;
-      const uint32_t off = static_cast<uint32_t>((e * kDPad + d0) * 4);
+  for (int i = 0; i < kBatch; ++i) {
+    const int it = gt + i * kGroup;
+    const int e = it >> 4, d = (it & 15) * 8;
+    const int el = e < kPartRows ? e : kZRow;
+    v[i][0] = __ldcg(reinterpret_cast<const float4*>(acc + el * kDPad + d));
+    v[i][1] = __ldcg(reinterpret_cast<const float4*>(acc + el * kDPad + d + 4));
+  }
+  const uint32_t bs = smem_u32(btile);
 #pragma unroll
-      for (int q = 0; q < cl::kMaxCluster; ++q)
-        if (q < C && it < r1 * 32 && e < kPartRows)
-          p[x][q] = q == me ? ld_shared_f4(part_s + off)
-                            : ld_shared_cluster_f4(mapa_shared(part_s + off, static_cast<uint32_t>(q)));
-    }
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const int it = base + x * nthr;
-      if (it >= r1 * 32) break;
-      const int e = it >> 5, d0 = (it & 31) * 4;
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
-      if (e < kPartRows) {
-#pragma unroll
-        for (int q = 0; q < cl::kMaxCluster; ++q) {
-          if (q < C) {
-            a[0] += p[x][q].x;
-            a[1] += p[x][q].y;
-            a[2] += p[x][q].z;
-            a[3] += p[x][q].w;
-          }
-        }
-        if (e < D) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (d0 + u < D) {
-              float* c = &sS[(e - r0) * ld + d0 + u];
-              if (has_S) a[u] += *c;
-              *c = a[u];
-            }
-          }
-        } else if (e == kZRow) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (d0 + u < D) {
-              if (has_z) a[u] += sZ[d0 + u];
-              sZ[d0 + u] = a[u];
-            }
-          }
-        }
-      }
-      uint2 w;
-      w.x = pack_bf16x2(a[0], a[1]);
-      w.y = pack_bf16x2(a[2], a[3]);
-      const uint32_t off = static_cast<uint32_t>((d0 >> 6) * (kPTileRows * 128) + e * 128 +
-                                                 ((((d0 & 63) >> 3) ^ (e & 7)) << 4) + (d0 & 7) * 2);
-      for (int q = 0; q < C; ++q) {
-        if (q == me)
-          st_shared_u2(ptile_s + off, w);
-        else
-          st_shared_cluster_u2(mapa_shared(ptile_s + off, static_cast<uint32_t>(q)), w);
-      }
+  for (int i = 0; i < kBatch; ++i) {
+    const int it = gt + i * kGroup;
+    const int e = it >> 4, d = (it & 15) * 8;
+    if (e >= kPartRows) v[i][0] = v[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint4 w;
+    w.x = pack_bf16x2(v[i][0].x, v[i][0].y);
+    w.y = pack_bf16x2(v[i][0].z, v[i][0].w);
+    w.z = pack_bf16x2(v[i][1].x, v[i][1].y);
+    w.w = pack_bf16x2(v[i][1].z, v[i][1].w);
+    st_shared_v4(bs + static_cast<uint32_t>((d >> 6) * (kPTileRows * 128) + e * 128 + ((((d & 63) >> 3) ^ (e & 7)) << 4)),
+                 w);
+    if (e >= r0 && e < ns_hi) {
+      *reinterpret_cast<float4*>(sS + (e - r0) * kDPad + d) = v[i][0];
+      *reinterpret_cast<float4*>(sS + (e - r0) * kDPad + d + 4) = v[i][1];
+    } else if (e == kZRow && share_has_z(r0, r1)) {
+      *reinterpret_cast<float4*>(sZ + d) = v[i][0];
+      *reinterpret_cast<float4*>(sZ + d + 4) = v[i][1];
     }
   }
 }
 
+// MMA issuer, phase 3: ReLU(Q_j) [P | z]^T for every resident tile, accumulators alternating.
+__device__ void mma_out(uint8_t* smem, const Bars3& b3, const Range& rg, bool two_atoms, uint32_t tmem,
+                        uint32_t* status) {
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, kPTileRows, false, false);
+  const int ksteps = two_atoms ? 8 : 4;
+  const uint32_t bbase = smem_u32(smem + kPartOff);
+  for (int j = 0; j < rg.n; ++j) {
+    const int a = j & 1;
+    if (!mbar_wait(&b3.qrelu[j], 0, status, 0x3520u | j)) break;
+    if (!mbar_wait(&b3.acce[a], ((j >> 1) & 1) ^ 1, status, 0x3530u | a)) break;
+    tc_fence_after();
+    const uint32_t qb = smem_u32(smem + j * kQSlot);
+    const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
+    for (int kk = 0; kk < ksteps; ++kk) {
+      const uint64_t ad = sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = sdesc_sw128(bbase + (kk >> 2) * (kPTileRows * 128) + (kk & 3) * 32, 16, 1024);
+      mma_bf16(dacc, ad, bd, kIdescO, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&b3.accf[a]);
+  }
+  mma_commit(b3.done);
+  mbar_wait(b3.done, 0, status, 0x35F0u);
+}
+
+// Epilogue of every tile for one warp: TMEM lanes 32q.. (tokens), output columns 64h..64h+63;
+// numerator / (denominator + eps) in bf16 into the tile's own Q slot (rows 32q.. of atom h), then
+// a TMA store of those rows (16-row box where the range ends inside the warp's 32 rows).
+__device__ void epilogue(uint8_t* smem, const Bars3& b3, const Maps& m, const Range& rg, int bh, uint32_t tmem, int q,
+                         int h, int lane, float eps, uint32_t* status) {
+  for (int j = 0; j < rg.n; ++j) {
+    const int a = j & 1;
+    if (!warp_all(mbar_wait(&b3.accf[a], (j >> 1) & 1, status, 0x3600u | a))) break;
+    tc_fence_after();
+    const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * 256);
+    uint32_t dr;
+    uint32_t rr[2][32];
+    tmem_ld_x1(ta + kZRow, dr);
+    tmem_ld_x32(ta + h * 64, rr[0]);
+    tmem_ld_x32(ta + h * 64 + 32, rr[1]);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b3.acce[a]);
+    const float inv = __frcp_rn(__uint_as_float(dr) + eps);
+    uint8_t* ob = smem + j * kQSlot + h * kAtomBytes + q * (32 * 128);
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 0]) * inv, __uint_as_float(rr[cc][8 * mm + 1]) * inv);
+        w.y = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 2]) * inv, __uint_as_float(rr[cc][8 * mm + 3]) * inv);
+        w.z = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 4]) * inv, __uint_as_float(rr[cc][8 * mm + 5]) * inv);
+        w.w = pack_bf16x2(__uint_as_float(rr[cc][8 * mm + 6]) * inv, __uint_as_float(rr[cc][8 * mm + 7]) * inv);
+        const int chunk = cc * 4 + mm;
+        *reinterpret_cast<uint4*>(ob + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int tok0 = rg.tok0(j), rows = rg.rows(j), valid = rows - q * 32;
+      if (valid > 0) {
+        if (valid >= 32 || tok0 + rows >= rg.N)  // whole slice, or clipped at the head's end by the map
+          tma_store_4d(m.o, ob, h * 64, tok0 + q * 32, 0, bh);
+        else                                     // the range ends 16 rows into the slice
+          tma_store_4d(m.o16, ob, h * 64, tok0 + q * 32, 0, bh);
+      }
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait_all();
+}
+}  // namespace cl
+
 __global__ void __launch_bounds__(kThreads, 1)
-    cluster_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
-                        const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
-                        const __grid_constant__ CUtensorMap q_main, const __grid_constant__ CUtensorMap q_last,
-                        const __grid_constant__ CUtensorMap o_main, const __grid_constant__ CUtensorMap o_last,
-                        const Geom geo, const float* S_in, const float* z_in, float* S_out, float* z_out,
-                        const float eps, uint32_t* status) {
+    cluster_bf16_kernel(const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+                        const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap o_map,
+                        const __grid_constant__ CUtensorMap k16_map, const __grid_constant__ CUtensorMap v16_map,
+                        const __grid_constant__ CUtensorMap q16_map, const __grid_constant__ CUtensorMap o16_map,
+                        const Geom geo, float* __restrict__ accum, const float* S_in, const float* z_in,
+                        float* S_out, float* z_out, const float eps, uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + cl::kBarOff);
   const st::Bars sb = st::bars_at(barmem);
-  const ot::Bars ob = ot::bars_at(barmem + st::kNumBars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + st::kNumBars + ot::kNumBars);
-  volatile int4* ring = reinterpret_cast<volatile int4*>(barmem + st::kNumBars + ot::kNumBars + 2);  // 16-byte aligned
+  const cl::Bars3 b3 = cl::bars3_at(barmem + st::kNumBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + cl::kNumBars);
   float* part = reinterpret_cast<float*>(smem + cl::kPartOff);
   float* sS = reinterpret_cast<float*>(smem + cl::kScratchOff);
   float* sZ = reinterpret_cast<float*>(smem + cl::kScratchZOff);
@@ -1395,82 +1647,101 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int C = static_cast<int>(gridDim.x) / geo.BH;  // cluster size (grid = B*H clusters of C CTAs)
   const int bh = static_cast<int>(cluster_id_x());
   const int r = static_cast<int>(cluster_ctarank());
-  const long long tb = static_cast<long long>(bh) * geo.tph + static_cast<long long>(r) * geo.tph / C;
-  const long long te = static_cast<long long>(bh) * geo.tph + static_cast<long long>(r + 1) * geo.tph / C;
-  const int r0 = 4 * (r * (kPTileRows / 4) / C), r1 = 4 * ((r + 1) * (kPTileRows / 4) / C);  // whole quads
+  const int units = (geo.N + cl::kUnit - 1) / cl::kUnit;
+  cl::Range rg;
+  rg.row0 = r * units / C * cl::kUnit;
+  rg.row1 = (r + 1) * units / C * cl::kUnit;
+  if (rg.row1 > geo.N) rg.row1 = geo.N;
+  rg.n = (rg.row1 - rg.row0 + kTile - 1) / kTile;
+  rg.N = geo.N;
+  const int r0 = 4 * (r * (kPTileRows / 4) / C), r1 = 4 * ((r + 1) * (kPTileRows / 4) / C);  // cache share rows
   const bool two_atoms = geo.D > 64;
-  const Maps4 mkv{&k_main, &k_last, &v_main, &v_last};
-  const Maps4 mqo{&q_main, &q_last, &o_main, &o_last};
+  const cl::Maps mp{&k_map, &v_map, &q_map, &o_map, &k16_map, &v16_map, &q16_map, &o16_map};
+  float* acc = accum + static_cast<size_t>(bh) * kPartRows * kDPad;
   if (threadIdx.x == 0) {
     st::init_bars(sb);
-    ot::init_bars(ob, two_atoms);
+    for (int j = 0; j < cl::kMaxTiles; ++j) {
+      mbar_init(&b3.qfull[j], 1);
+      mbar_init(&b3.qrelu[j], 4);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&b3.accf[a], 1);
+      mbar_init(&b3.acce[a], two_atoms ? 8 : 4);
+    }
+    mbar_init(b3.done, 1);
     fence_mbar_init();
   }
   st::init_smem(smem, two_atoms, kThreads);
   if (warp == kWarpProducer && lane == 0) {
-    prefetch_maps(mkv);
-    prefetch_maps(mqo);
+    prefetch_tmap(&k_map);
+    prefetch_tmap(&v_map);
+    prefetch_tmap(&q_map);
+    prefetch_tmap(&o_map);
+    prefetch_tmap(&k16_map);
+    prefetch_tmap(&v16_map);
+    prefetch_tmap(&q16_map);
+    prefetch_tmap(&o16_map);
   }
   const uint32_t tmem = persistent_setup(tmem_slot, warp);
-  griddep_wait();  // the previous kernel in the stream may still write q, k, v or the cache
+  griddep_wait();  // the previous kernel in the stream may still write q, k, v, the cache or the workspace
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  // phase 1: this rank's partial state; the epilogue warps first fetch the cache share
-  if (warp == kWarpProducer) {
-    if (lane == 0) st::produce(smem, sb, mkv, geo, tb, te, two_atoms, false, status);
-  } else if (warp >= 4 && warp < 8) {
-    st::relu_role(smem, sb, tb, te, two_atoms, threadIdx.x - 128, lane, status);
-  } else if (warp == kWarpMma) {
-    if (lane == 0) st::mma_role(smem, sb, geo, tb, te, tmem, status);
+  if (warp < 4) {
+    // phase 1 for the epilogue warps: zero this rank's share of the accumulator, fetch its share of
+    // the incoming cache, publish the zeroing (B1), then drain and reduce
+    const int z1 = r1 < kPartRows ? r1 : kPartRows;
+    for (int i = threadIdx.x; i < (z1 > r0 ? (z1 - r0) * (kDPad / 4) : 0); i += 128)
+      reinterpret_cast<float4*>(acc + r0 * kDPad)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    cl::load_cache_share(geo, S_in, z_in, bh, r0, r1, sS, sZ, threadIdx.x);
+    cl::arrive_release();  // B1
+    fence_proxy_async_smem();  // the cache share in sS / sZ -> its bulk reduction (async proxy)
+    cl::named_sync(1, 128);
+    cl::drain_reduce(sb, geo, tmem, warp, lane, part, acc, S_in != nullptr, z_in != nullptr, r0, r1, sS, sZ, status);
+    cl::arrive_release();  // B2: this rank's reductions are complete
+  } else if (warp < 8) {
+    cl::arrive_relaxed();  // B1 (nothing to publish)
+    st::relu_role(smem, sb, 0, rg.n, two_atoms, threadIdx.x - 128, lane, status);
+    cl::wait_acquire();
+    cl::arrive_relaxed();  // B2
+    // ReLU of each Q tile as it lands
+    for (int j = 0; j < rg.n; ++j) {
+      if (!warp_all(mbar_wait(&b3.qfull[j], 0, status, 0x3200u | j))) break;
+      relu_tile_inplace(smem + j * cl::kQSlot, (two_atoms ? cl::kQSlot : kAtomBytes) / 16, threadIdx.x - 128);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b3.qrelu[j]);
+    }
   } else {
-    combine_load_cache_q(geo, S_in, z_in, bh, r0, r1, sS, sZ, threadIdx.x, 128);
-    cl_drain_partial(sb, tmem, warp, lane, part, status);
+    cl::arrive_relaxed();  // B1
+    if (lane == 0) {
+      if (warp == kWarpProducer)
+        cl::produce(smem, sb, b3, mp, rg, bh, two_atoms, status);
+      else
+        cl::mma_state(smem, sb, rg, tmem, status);
+    }
+    __syncwarp();
+    cl::wait_acquire();
+    cl::arrive_relaxed();  // B2
   }
-  __syncthreads();
-
-  // phase 2: Q stages fill while the cluster exchanges the partial states. The Q loads are issued
-  // after the first cluster barrier: issued before it, they delayed its release by about 1 us.
-  const int pre = static_cast<int>(te - tb < ot::kStages ? te - tb : ot::kStages);  // Q tiles prefilled
-  const ot::Seq sq{tb, te, 0, 0, nullptr, ring};
-  cluster_arrive_release();
-  cluster_wait_acquire();
-  if (warp == kWarpProducer && lane == 0) ot::prefill(smem, ob, mqo, geo, sq, two_atoms);
-  // The ReLU warps rewrite the prefilled Q tiles that have already landed while the other warps
-  // combine (the combine is bound by distributed-shared-memory bandwidth, not by its thread count);
-  // tiles still in flight are left to phase 3 so that the second barrier never waits for Q.
-  int relu_done = 0;
-  if (warp >= 4 && warp < 8) {
-    while (relu_done < pre && warp_all(mbar_try_wait(&ob.qfull[relu_done], 0)) &&
-           ot::relu_q(smem, ob, sq, relu_done, two_atoms, threadIdx.x - 128, lane, status) > 0)
-      ++relu_done;
-  } else {
-    const int tid = warp < 4 ? static_cast<int>(threadIdx.x) : 128 + (warp - kWarpProducer) * 32 + lane;
-    cl_combine(geo, smem_u32(part), smem_u32(smem + ot::kBOff), C, r, S_in != nullptr, z_in != nullptr, r0, r1, sS,
-               sZ, tid, 192);
+  if (warp < 4 || warp >= 8) {
+    cl::wait_acquire();  // B2: the head's summed state is in L2
+    const int gt = warp < 4 ? static_cast<int>(threadIdx.x) : 128 + (warp - kWarpProducer) * 32 + lane;
+    cl::read_back(geo, acc, smem + cl::kPartOff, r0, r1, sS, sZ, gt);
+    fence_proxy_async_smem();  // the B tile -> tcgen05.mma (async proxy)
+    cl::named_sync(2, 192);
+    tc_fence_after();
+    // the outgoing cache while the output runs (nothing in this launch reads it): warp 8
+    if (warp == kWarpProducer) cl::store_cache_share(geo, S_out, z_out, bh, r0, r1, sS, sZ, lane, 32);
   }
-  fence_proxy_async_all();
-  cluster_arrive_release();
-  cluster_wait_acquire();
-  fence_proxy_async_all();  // the prefix tile written by the cluster -> tcgen05.mma reads (async proxy)
-  tc_fence_after();
-
-  // phase 3: output of this rank's tiles against the resident prefix tile. The partial states are
-  // no longer read by any rank, so their memory becomes double-buffered output staging. (After a
-  // failed wait anywhere in the grid every later wait returns at once, so phase 3 runs regardless.)
-  const ot::Staging sg{smem + cl::kPartOff, 2};
-  if (warp == kWarpProducer) {
-    if (lane == 0) ot::produce(smem, ob, mqo, geo, sq, pre, two_atoms, nullptr, nullptr, 0, status);
-  } else if (warp >= 4 && warp < 8) {
-    ot::relu_epi_role(smem, sg, ob, mqo, geo, sq, relu_done, two_atoms, tmem, warp, lane, eps, status);
-  } else if (warp == kWarpMma) {
-    if (lane == 0) ot::mma_role(smem, ob, geo, sq, two_atoms, tmem, status);
-  } else {
-    ot::epilogue_role(sg, ob, mqo, geo, sq, tmem, warp, lane, eps, status);
+  // phase 3: output MMAs and epilogues
+  if (warp < 4) {
+    cl::epilogue(smem, b3, mp, rg, bh, tmem, warp, 0, lane, eps, status);
+  } else if (warp < 8) {
+    cl::wait_acquire();  // B2 (taken here so that the Q ReLU above never waits for it)
+    if (two_atoms) cl::epilogue(smem, b3, mp, rg, bh, tmem, warp & 3, 1, lane, eps, status);
+  } else if (warp == kWarpMma && lane == 0) {
+    cl::mma_out(smem, b3, rg, two_atoms, tmem, status);
   }
-  // the outgoing cache last: nothing in this launch reads it, and its stores drain with the output
-  // (lanes 1..31 of the producer and MMA warps wait for lane 0 first, so they do not compete with it)
-  __syncwarp();
-  combine_store_cache_q(geo, S_out, z_out, bh, r0, r1, sS, sZ, threadIdx.x, kThreads);
   persistent_teardown(tmem, warp);
 }
 
@@ -1710,17 +1981,20 @@ int cluster_size(const Geom& g, int sm_count) {
     }
     known[dev] = true;
   }
+  // every rank gets at least one 16-row unit and at most kMaxTiles tiles of rows
+  const int units = cdiv(g.N, cl::kUnit);
   for (int c = cl::kMaxCluster; c >= cl::kMinCluster; --c) {
-    if (c > g.tph || max_active[dev][c] < g.BH) continue;
+    if (g.nblk != 1 || units < c || cdiv(units, c) * cl::kUnit > cl::kMaxTiles * kTile) continue;
+    if (max_active[dev][c] < g.BH) continue;
     if (static_cast<long long>(g.BH) * c * 4 < static_cast<long long>(sm_count) * 3) continue;
     return c;
   }
   return 0;
 }
 
-cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
-                                const Geom& g, int C, const float* S_in, const float* z_in, float* S_out,
-                                float* z_out, float eps, uint32_t* status, cudaStream_t s) {
+cudaError_t launch_cluster_bf16(const ClusterMaps& m, const Geom& g, int C, float* accum, const float* S_in,
+                                const float* z_in, float* S_out, float* z_out, float eps, uint32_t* status,
+                                cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(g.BH * C));
   cfg.blockDim = dim3(kThreads);
@@ -1735,8 +2009,8 @@ cudaError_t launch_cluster_bf16(const BlockMaps& k, const BlockMaps& v, const Bl
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, cluster_bf16_kernel, k.main, k.last, v.main, v.last, q.main, q.last, o.main,
-                            o.last, g, S_in, z_in, S_out, z_out, eps, status);
+  return cudaLaunchKernelEx(&cfg, cluster_bf16_kernel, m.k, m.v, m.q, m.o, m.k16, m.v16, m.q16, m.o16, g, accum, S_in,
+                            z_in, S_out, z_out, eps, status);
 }
 
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
