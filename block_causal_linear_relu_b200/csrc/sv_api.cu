@@ -279,6 +279,9 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
       SV_TRY(encode_map(&cm.v16, v, g.N, 1, g, 16));
       SV_TRY(encode_map(&cm.q16, q, g.N, 1, g, 16));
       SV_TRY(encode_map(&cm.o16, o, g.N, 1, g, 16));
+      SV_TRY(encode_map(&cm.k64, k, g.N, 1, g, 64));
+      SV_TRY(encode_map(&cm.v64, v, g.N, 1, g, 64));
+      SV_TRY(encode_map(&cm.q64, q, g.N, 1, g, 64));
       prof_mark(0, stream);
       e = sv::launch_cluster_bf16(cm, g, C, partials, S_in, z_in, S_out, z_out, eps, status, stream);
       if (e != cudaSuccess) return cuda_fail(e, "cluster kernel launch");

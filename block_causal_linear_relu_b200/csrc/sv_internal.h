@@ -39,11 +39,11 @@ cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const Bloc
                               uint32_t* status, cudaStream_t st);
 // bf16, whole sequence in one block, few heads: one thread-block cluster of C CTAs per head, whose
 // ranks split the head's rows in 16-row units. Maps of the one-block [BH, N, D] tensors: k, v, q
-// with 128-row boxes, o with 32-row store boxes, and the same four with 16-row boxes. The head's
-// summed state is reduced in `accum` (fp32 [BH][129][128] in the workspace).
+// with 128-row boxes, o with 32-row store boxes, the same four with 16-row boxes and k, v, q with
+// 64-row boxes. The head's summed state is reduced in `accum` (fp32 [BH][129][128] in the workspace).
 // cluster_size returns the C to use for this geometry (0: use launch_fused_bf16 instead).
 struct ClusterMaps {
-  CUtensorMap k, v, q, o, k16, v16, q16, o16;
+  CUtensorMap k, v, q, o, k16, v16, q16, o16, k64, v64, q64;
 };
 int cluster_size(const Geom& g, int sm_count);
 cudaError_t launch_cluster_bf16(const ClusterMaps& m, const Geom& g, int C, float* accum, const float* S_in,

@@ -1245,7 +1245,7 @@ constexpr int kShareRowsMax = (kPTileRows + kMinCluster - 1) / kMinCluster;
 constexpr int kScratchOff = kRegion;                 // cache share [row][128] fp32 (S_in, then P)
 constexpr int kScratchZOff = kScratchOff + kShareRowsMax * kDPad * 4;
 constexpr int kBarOff = (kScratchZOff + kDPad * 4 + 127) / 128 * 128;
-constexpr int kNumBars = st::kNumBars + 2 * kMaxTiles + 5;
+constexpr int kNumBars = st::kNumBars + 2 * kMaxTiles + 7;
 constexpr int kSmem = kBarOff + 512 + 1024;
 static_assert(kNumBars * 8 + 8 <= 512, "barrier area");
 static_assert(kSmem <= 227 * 1024, "cluster kernel shared memory");
@@ -1256,9 +1256,12 @@ struct Bars3 {            // phase 3
   uint64_t* accf;         // [2] output accumulator holds a tile
   uint64_t* acce;         // [2] output accumulator drained
   uint64_t* done;
+  uint64_t* kvi;          // the producer has issued the first K/V stages
+  uint64_t* rb;           // the summed state has landed in shared memory (read-back copy)
 };
 __device__ __forceinline__ Bars3 bars3_at(uint64_t* p) {
-  return Bars3{p, p + kMaxTiles, p + 2 * kMaxTiles, p + 2 * kMaxTiles + 2, p + 2 * kMaxTiles + 4};
+  return Bars3{p, p + kMaxTiles, p + 2 * kMaxTiles, p + 2 * kMaxTiles + 2, p + 2 * kMaxTiles + 4,
+               p + 2 * kMaxTiles + 5, p + 2 * kMaxTiles + 6};
 }
 
 // Tiles of one rank: tile j starts at row tok0(j) of the head and holds rows(j) rows.
@@ -1283,6 +1286,9 @@ struct Maps {
   const CUtensorMap* v16;
   const CUtensorMap* q16;
   const CUtensorMap* o16;
+  const CUtensorMap* k64;  // 64-row boxes
+  const CUtensorMap* v64;
+  const CUtensorMap* q64;
 };
 
 // non-aligned cluster barrier halves: each thread arrives and waits at its own point
@@ -1299,21 +1305,26 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src,
 }
 
 // Loads rows(j) rows of one [BH, N, D] tensor at (tok0, bh) into `dst` (128-row tile layout, one or
-// two 16 KB atoms); returns the bytes the barrier must expect.
-__device__ __forceinline__ uint32_t load_rows(uint8_t* dst, const CUtensorMap* m128, const CUtensorMap* m16,
-                                              uint64_t* bar, const Range& rg, int j, int bh, bool two_atoms,
-                                              uint64_t pol) {
+// two 16 KB atoms): one whole box, or for a range ending inside the tile one 64-row box and 16-row
+// boxes for the rest (each copy instruction holds the producer for a while, so few and large).
+__device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m128, const CUtensorMap* m64,
+                                          const CUtensorMap* m16, uint64_t* bar, const Range& rg, int j, int bh,
+                                          bool two_atoms, uint64_t pol) {
   const int tok0 = rg.tok0(j);
   const int na = two_atoms ? 2 : 1;
   if (!rg.boxed16(j)) {
     for (int a = 0; a < na; ++a) tma_load_4d(dst + a * kAtomBytes, m128, bar, 64 * a, tok0, 0, bh, pol);
-    return static_cast<uint32_t>(na * kAtomBytes);
+    return;
   }
   const int nb = rg.rows(j) / kUnit;
-  for (int u = 0; u < nb; ++u)
+  int u = 0;
+  if (nb >= 4) {
+    for (int a = 0; a < na; ++a) tma_load_4d(dst + a * kAtomBytes, m64, bar, 64 * a, tok0, 0, bh, pol);
+    u = 4;
+  }
+  for (; u < nb; ++u)
     for (int a = 0; a < na; ++a)
       tma_load_4d(dst + a * kAtomBytes + u * (kUnit * 128), m16, bar, 64 * a, tok0 + u * kUnit, 0, bh, pol);
-  return static_cast<uint32_t>(nb * na * kUnit * 128);
 }
 
 // Producer, phase 1: the rank's K and V tiles through the three stages; then, once every state
@@ -1324,22 +1335,27 @@ __device__ void produce(uint8_t* smem, const st::Bars& b, const Bars3& b3, const
   int j = 0;
   for (; j < rg.n; ++j) {
     const int s = j % st::kStages;
-    if (!mbar_wait(&b.empty[s], ((j / st::kStages) & 1) ^ 1, status, 0x3100u | s)) return;
+    if (j == st::kStages) mbar_arrive(b3.kvi);  // the first stages are in flight
+    if (!mbar_wait(&b.empty[s], ((j / st::kStages) & 1) ^ 1, status, 0x3100u | s)) {
+      if (j < st::kStages) mbar_arrive(b3.kvi);
+      return;
+    }
     uint8_t* stg = smem + s * st::kStageBytes;
     // both expect_tx before either copy, so the phase cannot complete early
     const int nb = rg.boxed16(j) ? rg.rows(j) / kUnit : 0;
     const uint32_t per = nb ? static_cast<uint32_t>(nb * kUnit * 128) : static_cast<uint32_t>(kAtomBytes);
     mbar_expect_tx(&b.full[s], (two_atoms ? 4u : 2u) * per);
-    load_rows(stg, m.k, m.k16, &b.full[s], rg, j, bh, two_atoms, pol);
-    load_rows(stg + st::kKBytes, m.v, m.v16, &b.full[s], rg, j, bh, two_atoms, pol);
+    load_rows(stg, m.k, m.k64, m.k16, &b.full[s], rg, j, bh, two_atoms, pol);
+    load_rows(stg + st::kKBytes, m.v, m.v64, m.v16, &b.full[s], rg, j, bh, two_atoms, pol);
   }
+  if (rg.n <= st::kStages) mbar_arrive(b3.kvi);
   for (int i = (rg.n > st::kStages ? rg.n - st::kStages : 0); i < rg.n; ++i)
     if (!mbar_wait(&b.empty[i % st::kStages], (i / st::kStages) & 1, status, 0x3180u)) return;
   for (int i = 0; i < rg.n; ++i) {
     const int nb = rg.boxed16(i) ? rg.rows(i) / kUnit : 0;
     const uint32_t per = nb ? static_cast<uint32_t>(nb * kUnit * 128) : static_cast<uint32_t>(kAtomBytes);
     mbar_expect_tx(&b3.qfull[i], (two_atoms ? 2u : 1u) * per);
-    load_rows(smem + i * kQSlot, m.q, m.q16, &b3.qfull[i], rg, i, bh, two_atoms, pol);
+    load_rows(smem + i * kQSlot, m.q, m.q64, m.q16, &b3.qfull[i], rg, i, bh, two_atoms, pol);
   }
 }
 
@@ -1463,9 +1479,9 @@ __device__ void store_cache_share(const Geom& geo, float* __restrict__ S_out, fl
 // key feature d) is drained into the partial [e][d] in shared memory, and thread 0 adds each
 // drained half to the accumulator with a bulk reduction. Every thread of the four warps passes both
 // named barriers whatever happened before.
-__device__ void drain_reduce(const st::Bars& b, const Geom& geo, uint32_t tmem, int warp, int lane, float* part,
-                             float* acc, bool has_S, bool has_z, int r0, int r1, const float* sS, const float* sZ,
-                             uint32_t* status) {
+__device__ void drain_reduce(const st::Bars& b, const Geom& geo, uint32_t tmem, int warp, int lane, int rank,
+                             float* part, float* acc, bool has_S, bool has_z, int r0, int r1, const float* sS,
+                             const float* sZ, uint32_t* status) {
   const int d = warp * 32 + lane;
   const bool ok = warp_all(mbar_wait(&b.accf[0], 0, status, 0x3400u));
   wait_acquire();  // B1: every rank has zeroed its share of the accumulator
@@ -1479,14 +1495,17 @@ __device__ void drain_reduce(const st::Bars& b, const Geom& geo, uint32_t tmem, 
   if (ok) tc_fence_after();
   const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const uint32_t ps = smem_u32(part) + static_cast<uint32_t>(d * 4);
+  // ranks of odd index drain and reduce the second half first, so that the head's ranks do not
+  // all add into the same rows of the accumulator at the same time
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = hh ^ (rank & 1);
     if (ok) {
       uint32_t rr[2][32];
       uint32_t zr = 0;
       tmem_ld_x32(ta + h * 64, rr[0]);
       tmem_ld_x32(ta + h * 64 + 32, rr[1]);
-      if (h == 1) tmem_ld_x1(ta + 128, zr);
+      tmem_ld_x1(ta + 128, zr);
       tmem_wait_ld();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc)
@@ -1510,30 +1529,40 @@ __device__ void drain_reduce(const st::Bars& b, const Geom& geo, uint32_t tmem, 
   tc_fence_before();
 }
 
-// Read-back by the 192 threads of warps 0-3, 8 and 9 (index gt): the summed state P (fp32 [129][128]
-// in L2) into the bf16 B tile (rows 129..143 zero), and the rank's share of rows into sS / sZ for
-// the outgoing cache. Twelve (row, 8-feature) items per thread; the loads have no condition (rows
-// past z read row 128 and are zeroed afterwards) so that all 24 are in flight at once.
-__device__ void read_back(const Geom& geo, const float* acc, uint8_t* btile, int r0, int r1, float* __restrict__ sS,
-                          float* __restrict__ sZ, int gt) {
+// Read-back, after B2: thread 0 copies the summed state P (fp32 [129][128], in L2) into the partial
+// region with one bulk copy; then the 192 threads of warps 0-3, 8 and 9 (index gt) each take twelve
+// (row, 8-feature) items into registers, meet, and write them back in place as the bf16 B tile
+// (rows 129..143 zero) -- the tile overlaps the fp32 copy, hence the barrier between the two -- and
+// the rank's share of rows into sS / sZ for the outgoing cache.
+__device__ void read_back(const Geom& geo, const float* acc, const Bars3& b3, uint8_t* region, int r0, int r1,
+                          float* __restrict__ sS, float* __restrict__ sZ, int gt, uint32_t* status) {
   constexpr int kGroup = 192, kBatch = 12;
   static_assert(kGroup * kBatch == kPTileRows * 16, "one batch covers the B tile");
-  const int ns_hi = r0 + share_rows(geo, r0, r1);
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(b3.rb, kPartRows * kDPad * 4);
+    bulk_load(region, acc, kPartRows * kDPad * 4, b3.rb);
+  }
+  const bool ok = warp_all(mbar_wait(b3.rb, 0, status, 0x3700u));
+  const float* src = reinterpret_cast<const float*>(region);
   float4 v[kBatch][2];
 #pragma unroll
   for (int i = 0; i < kBatch; ++i) {
     const int it = gt + i * kGroup;
     const int e = it >> 4, d = (it & 15) * 8;
-    const int el = e < kPartRows ? e : kZRow;
-    v[i][0] = __ldcg(reinterpret_cast<const float4*>(acc + el * kDPad + d));
-    v[i][1] = __ldcg(reinterpret_cast<const float4*>(acc + el * kDPad + d + 4));
+    if (ok && e < kPartRows) {
+      v[i][0] = *reinterpret_cast<const float4*>(src + e * kDPad + d);
+      v[i][1] = *reinterpret_cast<const float4*>(src + e * kDPad + d + 4);
+    } else {
+      v[i][0] = v[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
-  const uint32_t bs = smem_u32(btile);
+  named_sync(2, kGroup);  // every fp32 value is in registers before the bf16 tile overwrites them
+  const int ns_hi = r0 + share_rows(geo, r0, r1);
+  const uint32_t bs = smem_u32(region);
 #pragma unroll
   for (int i = 0; i < kBatch; ++i) {
     const int it = gt + i * kGroup;
     const int e = it >> 4, d = (it & 15) * 8;
-    if (e >= kPartRows) v[i][0] = v[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
     uint4 w;
     w.x = pack_bf16x2(v[i][0].x, v[i][0].y);
     w.y = pack_bf16x2(v[i][0].z, v[i][0].w);
@@ -1631,7 +1660,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap o_map,
                         const __grid_constant__ CUtensorMap k16_map, const __grid_constant__ CUtensorMap v16_map,
                         const __grid_constant__ CUtensorMap q16_map, const __grid_constant__ CUtensorMap o16_map,
-                        const Geom geo, float* __restrict__ accum, const float* S_in, const float* z_in,
+                        const __grid_constant__ CUtensorMap k64_map, const __grid_constant__ CUtensorMap v64_map,
+                        const __grid_constant__ CUtensorMap q64_map, const Geom geo, float* __restrict__ accum, const float* S_in, const float* z_in,
                         float* S_out, float* z_out, const float eps, uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -1656,7 +1686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   rg.N = geo.N;
   const int r0 = 4 * (r * (kPTileRows / 4) / C), r1 = 4 * ((r + 1) * (kPTileRows / 4) / C);  // cache share rows
   const bool two_atoms = geo.D > 64;
-  const cl::Maps mp{&k_map, &v_map, &q_map, &o_map, &k16_map, &v16_map, &q16_map, &o16_map};
+  const cl::Maps mp{&k_map, &v_map, &q_map, &o_map, &k16_map, &v16_map, &q16_map, &o16_map,
+                    &k64_map, &v64_map, &q64_map};
   float* acc = accum + static_cast<size_t>(bh) * kPartRows * kDPad;
   if (threadIdx.x == 0) {
     st::init_bars(sb);
@@ -1669,6 +1700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&b3.acce[a], two_atoms ? 8 : 4);
     }
     mbar_init(b3.done, 1);
+    mbar_init(b3.kvi, 1);
+    mbar_init(b3.rb, 1);
     fence_mbar_init();
   }
   st::init_smem(smem, two_atoms, kThreads);
@@ -1681,6 +1714,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&v16_map);
     prefetch_tmap(&q16_map);
     prefetch_tmap(&o16_map);
+    prefetch_tmap(&k64_map);
+    prefetch_tmap(&v64_map);
+    prefetch_tmap(&q64_map);
   }
   const uint32_t tmem = persistent_setup(tmem_slot, warp);
   griddep_wait();  // the previous kernel in the stream may still write q, k, v, the cache or the workspace
@@ -1689,6 +1725,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     // phase 1 for the epilogue warps: zero this rank's share of the accumulator, fetch its share of
     // the incoming cache, publish the zeroing (B1), then drain and reduce
+    // their loads and stores wait until the producer's first K/V copies are issued: issued
+    // together, they held back the producer's copy instructions by about a microsecond
+    mbar_wait(b3.kvi, 0, status, 0x3050u);
     const int z1 = r1 < kPartRows ? r1 : kPartRows;
     for (int i = threadIdx.x; i < (z1 > r0 ? (z1 - r0) * (kDPad / 4) : 0); i += 128)
       reinterpret_cast<float4*>(acc + r0 * kDPad)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1696,7 +1735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cl::arrive_release();  // B1
     fence_proxy_async_smem();  // the cache share in sS / sZ -> its bulk reduction (async proxy)
     cl::named_sync(1, 128);
-    cl::drain_reduce(sb, geo, tmem, warp, lane, part, acc, S_in != nullptr, z_in != nullptr, r0, r1, sS, sZ, status);
+    cl::drain_reduce(sb, geo, tmem, warp, lane, r, part, acc, S_in != nullptr, z_in != nullptr, r0, r1, sS, sZ, status);
     cl::arrive_release();  // B2: this rank's reductions are complete
   } else if (warp < 8) {
     cl::arrive_relaxed();  // B1 (nothing to publish)
@@ -1726,9 +1765,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4 || warp >= 8) {
     cl::wait_acquire();  // B2: the head's summed state is in L2
     const int gt = warp < 4 ? static_cast<int>(threadIdx.x) : 128 + (warp - kWarpProducer) * 32 + lane;
-    cl::read_back(geo, acc, smem + cl::kPartOff, r0, r1, sS, sZ, gt);
+    cl::read_back(geo, acc, b3, smem + cl::kPartOff, r0, r1, sS, sZ, gt, status);
     fence_proxy_async_smem();  // the B tile -> tcgen05.mma (async proxy)
-    cl::named_sync(2, 192);
+    cl::named_sync(3, 192);
     tc_fence_after();
     // the outgoing cache while the output runs (nothing in this launch reads it): warp 8
     if (warp == kWarpProducer) cl::store_cache_share(geo, S_out, z_out, bh, r0, r1, sS, sZ, lane, 32);
@@ -2009,8 +2048,8 @@ cudaError_t launch_cluster_bf16(const ClusterMaps& m, const Geom& g, int C, floa
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, cluster_bf16_kernel, m.k, m.v, m.q, m.o, m.k16, m.v16, m.q16, m.o16, g, accum, S_in,
-                            z_in, S_out, z_out, eps, status);
+  return cudaLaunchKernelEx(&cfg, cluster_bf16_kernel, m.k, m.v, m.q, m.o, m.k16, m.v16, m.q16, m.o16, m.k64, m.v64,
+                            m.q64, g, accum, S_in, z_in, S_out, z_out, eps, status);
 }
 
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,
