@@ -347,6 +347,7 @@ def run_ours(args, rank: int, world: int):
         extras = {}
         for name, passes in EXTRA_PASSES.items():
             extras[name] = time_workload(name, passes, dev.index)
+        extras["720p_temporal_conv"] = time_conv(5, dev.index)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -479,6 +480,81 @@ def time_workload(name, passes: int, dev_index: int = 0):
 EXTRA_PASSES = {"480p_bidir": 200, "720p_stream": 5, "sv2_stack": 8, "720p_denoise": 4}
 
 
+def time_conv(passes: int, dev_index: int = 0):
+    """The block-causal temporal convolution (kernel width 3) on the 720p latent video the prefill
+    covers: x [1, 60, 920, 2560] bf16 (60 latent frames of 23 x 40 tokens, hidden 2560), blocks of 3
+    frames; one call over the whole sequence, and the same 20 blocks streamed with the carried frame.
+    Algorithmic bytes: read x and write y once (plus the carried frame read and written per block)."""
+    import torch
+
+    import block_causal_linear_relu_b200 as sv
+
+    dev = torch.device("cuda", dev_index)
+    hbm_gbs, _, _, _ = peaks()
+    B, T, S, C, Lb = 1, 60, 920, 2560, 3
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    xs = [torch.randn(B, T, S, C, device=dev, generator=gen).to(torch.bfloat16) for _ in range(2)]
+    w = torch.randn(C, 3, device=dev, generator=gen) * 0.5
+    b = torch.randn(C, device=dev, generator=gen) * 0.5
+    y = torch.empty_like(xs[0])
+    blocks = [[x[:, a:a + Lb].contiguous() for a in range(0, T, Lb)] for x in xs]
+    yb = torch.empty_like(blocks[0][0])
+    carry = torch.zeros(B, S, C, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    one_bytes = 2 * xs[0].numel() * 2
+    blk_bytes = 2 * blocks[0][0].numel() * 2 + 2 * carry.numel() * 2
+
+    def timed(fn, n):
+        fn(0)
+        torch.cuda.synchronize()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(dev.index) as clk:
+            a.record(stream)
+            for i in range(n):
+                fn(i)
+            e.record(stream)
+            torch.cuda.synchronize()
+        return a.elapsed_time(e) / n, clk.summary()
+
+    one_ms, clk1 = timed(lambda i: sv.sv_temporal_conv(xs[i % 2], w, Lb, bias=b, y=y, stream=stream), 10 * passes)
+    # the 20 blocks of both sequences captured once in a CUDA graph and replayed (a generation loop's
+    # way of issuing short calls): device time per block without the host's per-call work
+    nb = len(blocks[0])
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for seq in blocks:
+                for blk in seq:
+                    sv.sv_temporal_conv_step(blk, w, carry, bias=b, y=yb, stream=side)
+        graph.replay()
+        side.synchronize()
+        ga, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(dev.index) as clk2:
+            ga.record(side)
+            for _ in range(passes):
+                graph.replay()
+            ge.record(side)
+            side.synchronize()
+        blk_ms = ga.elapsed_time(ge) / (passes * 2 * nb)
+        clk2 = clk2.summary()
+    del graph
+    torch.cuda.synchronize()
+    return {
+        "workload": "block-causal temporal conv (width 3, depthwise) over x [1, 60, 920, 2560] bf16, blocks of 3 "
+                    "frames; one call, and 20 blocks streamed with the carried frame",
+        "one_shot": {"ms": one_ms, "alg_bytes": one_bytes, "hbm_gbs_alg": one_bytes / (one_ms / 1e3) / 1e9,
+                     "hbm_frac": one_bytes / (one_ms / 1e3) / 1e9 / hbm_gbs, "clocks": clk1},
+        "per_block": {"ms": blk_ms, "alg_bytes": blk_bytes, "hbm_gbs_alg": blk_bytes / (blk_ms / 1e3) / 1e9,
+                      "hbm_frac": blk_bytes / (blk_ms / 1e3) / 1e9 / hbm_gbs, "clocks": clk2},
+        "inputs": "two x tensors alternated (each 283 MB, more than L2); torch CUDA generator seed 0",
+        "timing": "CUDA events; one-shot: back-to-back calls on one stream, mean per call; per block: the 40 "
+                  "block calls captured in a CUDA graph and replayed, mean per call",
+    }
+
+
 def run_extra(args, name):
     """One configuration alone, as an informational JSON line (not the bench line)."""
     import torch
@@ -506,7 +582,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="leave the other configurations (480p, streaming, 2.0 stack, denoising) out of the line")
-    ap.add_argument("--workload", choices=["720p_prefill"] + sorted(EXTRA_WORKLOADS), default="720p_prefill",
+    ap.add_argument("--workload", choices=["720p_prefill", "720p_temporal_conv"] + sorted(EXTRA_WORKLOADS),
+                    default="720p_prefill",
                     help="the bench line is 720p_prefill; the others print an informational timing line")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H (profiling captures of a smaller case only; not a bench line)")
@@ -522,6 +599,12 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload == "720p_temporal_conv":
+        import torch
+        torch.cuda.set_device(0)
+        print(json.dumps({"workload": "720p_temporal_conv", "impl": "ours", **time_conv(max(1, args.steps // 20))}),
+              flush=True)
+        return 0
     if args.workload != "720p_prefill":
         return run_extra(args, args.workload)
     if world > 1:

@@ -26,5 +26,7 @@ from ._native import (  # noqa: F401
     sv_linattn_fwd,
     sv_profile_events,
     sv_selftest_wait_timeout,
+    sv_temporal_conv,
+    sv_temporal_conv_step,
     workspace_bytes,
 )

@@ -26,8 +26,8 @@ SV_OP_LINATTN_FWD, SV_OP_BLOCK_STATE_UPDATE, SV_OP_BLOCK_CAUSAL_ATTN, SV_OP_CACH
 EXPORTS = (
     "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_workspace_set_mirror", "sv_linattn_fwd",
     "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_cache_step_noalloc",
-    "sv_cache_step_noalloc_status", "sv_profile_events", "sv_last_error", "sv_selftest_wait_timeout",
-    "sv_version",
+    "sv_cache_step_noalloc_status", "sv_temporal_conv", "sv_temporal_conv_step", "sv_profile_events",
+    "sv_last_error", "sv_selftest_wait_timeout", "sv_version",
 )
 
 
@@ -73,6 +73,10 @@ def load() -> ctypes.CDLL:
         lib.sv_cache_step_noalloc.restype = i
         lib.sv_cache_step_noalloc_status.argtypes = [vp, u32p]
         lib.sv_cache_step_noalloc_status.restype = i
+        lib.sv_temporal_conv.argtypes = [vp, vp, i, i, i, i, i, vp, vp, i, vp]
+        lib.sv_temporal_conv.restype = i
+        lib.sv_temporal_conv_step.argtypes = [vp, vp, i, i, i, i, vp, vp, vp, i, i, vp]
+        lib.sv_temporal_conv_step.restype = i
         lib.sv_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
         lib.sv_profile_events.restype = i
         lib.sv_last_error.argtypes = []
@@ -282,3 +286,36 @@ def sv_block_state_update(k, v, S, z, ws: Workspace | None = None, stream=None):
     _check(load().sv_block_state_update(_ptr(k), _ptr(v), B, H, N, D, _dt(k), _ptr(S), _ptr(z), ws.ptr, ws.nbytes,
                                         _stream(stream)))
     return S, z
+
+
+def _conv_args(x, w, bias):
+    if not x.is_cuda or x.dim() != 4 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor [B, T, S, C]")
+    C = x.shape[3]
+    if w.dtype != torch.float32 or tuple(w.shape) != (C, 3) or not w.is_contiguous() or w.device != x.device:
+        raise ValueError("w must be a contiguous float32 [C, 3] tensor on x's device")
+    if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (C,) or bias.device != x.device):
+        raise ValueError("bias must be a float32 [C] tensor on x's device")
+
+
+def sv_temporal_conv(x, w, frames_per_block: int, bias=None, y=None, stream=None):
+    """Block-causal temporal convolution over x [B, T, S, C] (kernel width 3); returns y."""
+    _conv_args(x, w, bias)
+    y = torch.empty_like(x) if y is None else y
+    B, T, S, C = x.shape
+    _check(load().sv_temporal_conv(_ptr(x), _ptr(y), B, T, S, C, int(frames_per_block), _ptr(w), _ptr(bias), _dt(x),
+                                   _stream(stream)))
+    return y
+
+
+def sv_temporal_conv_step(x, w, carry, commit: bool = True, bias=None, y=None, stream=None):
+    """One block x [B, T, S, C] of a stream with the previous block's last frame in carry [B, S, C]
+    (zeros before the first block); carry takes x's last frame if commit. Returns y."""
+    _conv_args(x, w, bias)
+    B, T, S, C = x.shape
+    if carry.dtype != x.dtype or tuple(carry.shape) != (B, S, C) or not carry.is_contiguous():
+        raise ValueError("carry must be a contiguous [B, S, C] tensor of x's dtype")
+    y = torch.empty_like(x) if y is None else y
+    _check(load().sv_temporal_conv_step(_ptr(x), _ptr(y), B, T, S, C, _ptr(w), _ptr(bias), _ptr(carry),
+                                        1 if commit else 0, _dt(x), _stream(stream)))
+    return y

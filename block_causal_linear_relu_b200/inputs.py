@@ -62,3 +62,15 @@ def draw_qkv(shape, seed: int, dtype: str = BF16, scale: float = 1.0):
 def to_f64(x: np.ndarray, dtype: str) -> np.ndarray:
     """Storage form -> float64 values exactly as the kernels see them."""
     return bf16_bits_to_f64(x) if dtype == BF16 else np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+def draw_conv(shape, seed: int, dtype: str = BF16):
+    """Inputs of the temporal convolution: x ~ N(0, 1) of `shape` [B, T, S, C] in storage form, then
+    fp32 weights w [C, 3] ~ N(0, 1/4) and bias [C] ~ N(0, 1/4) (synthetic: the pages give none), all
+    from one seeded generator in that order."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(shape, dtype=np.float32)
+    C = shape[-1]
+    w = (rng.standard_normal((C, 3), dtype=np.float32) * np.float32(0.5)).astype(np.float32)
+    b = (rng.standard_normal((C,), dtype=np.float32) * np.float32(0.5)).astype(np.float32)
+    return (f32_to_bf16_bits(x) if dtype == BF16 else x), w, b

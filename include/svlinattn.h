@@ -165,6 +165,30 @@ sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, voi
  * the word in *code if given). Allocates nothing. */
 sv_status sv_cache_step_noalloc_status(sv_stream_t stream, uint32_t* code);
 
+/* Block-causal temporal convolution of the causal Mix-FFN (talk, causal FFN with temporal conv
+ * passage: a zero token is padded between two blocks so that block 1 cannot see block 2, and block
+ * 2 takes block 1's last token as its first token so that it sees block 1; the padding and the
+ * carried token are dropped after the convolution; the model-family page places a one-dimensional
+ * temporal convolution inside the Mix-FFN). The pages give neither the width nor the weights; this
+ * library reads the passage as a depthwise convolution along time with a centred kernel of width 3
+ * (one padding token, one carried token), in cross-correlation order:
+ *     y[t] = w[c][0] * x[t-1] + w[c][1] * x[t] + w[c][2] * x[t+1] * [blk(t+1) == blk(t)] + bias[c],
+ * blk(t) = floor(t / frames_per_block), x[-1] = 0; the last block may be shorter.
+ * x, y: DEVICE pointers to contiguous [B, T, S, C] tensors (T latent frames of S tokens, C channels,
+ * C fastest), element type dt, 16-byte aligned; C a multiple of 8 (bf16) or 4 (fp32). y may equal x.
+ * w: DEVICE fp32 [C][3]; bias: DEVICE fp32 [C] or NULL. Computed in fp32, rounded once to dt. */
+sv_status sv_temporal_conv(const void* x, void* y, int B, int T, int S, int C, int frames_per_block, const float* w,
+                           const float* bias, sv_dtype dt, sv_stream_t stream);
+
+/* One block of a stream through the same convolution: the T frames of x form one block; carry
+ * (DEVICE [B, S, C] of dt, 16-byte aligned, zeros before the first block) is the previous block's
+ * last frame, seen by frame 0 as its left neighbour; the block's last frame has the padding zero on
+ * its right. If commit != 0, carry then receives x's last frame (in place). Memory kept between
+ * blocks: carry only, whatever the number of blocks. Block by block this equals sv_temporal_conv of
+ * the whole sequence (talk, causal FFN with temporal conv passage). */
+sv_status sv_temporal_conv_step(const void* x, void* y, int B, int T, int S, int C, const float* w, const float* bias,
+                                void* carry, int commit, sv_dtype dt, sv_stream_t stream);
+
 /* Optional timing hook for benchmarks. With events != NULL (n == 4 cudaEvent_t handles owned by
  * the caller), the calling thread's following forward calls (sv_linattn_fwd, sv_block_causal_attn,
  * sv_cache_step) record events[0] before the state-reduction kernel, events[1] after it,
