@@ -348,6 +348,7 @@ def run_ours(args, rank: int, world: int):
         for name, passes in EXTRA_PASSES.items():
             extras[name] = time_workload(name, passes, dev.index)
         extras["720p_temporal_conv"] = time_conv(5, dev.index)
+        extras["sv2_projections"] = time_proj(20, dev.index)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -555,6 +556,62 @@ def time_conv(passes: int, dev_index: int = 0):
     }
 
 
+def time_proj(reps: int, dev_index: int = 0):
+    """The projections of one SANA-Video 2.0-shaped layer: x [2, 10120, 2560] bf16 -> ReLU(q), ReLU(k), v
+    [2, 20, 10120, 128] (W_qkv [7680, 2560]) and o [2, 20, 10120, 128] -> y [2, 10120, 2560] (W_o [2560,
+    2560]). Tensor-bound: flops 2 * M * N * K; the roofline is the measured cuBLAS bf16 rate. cuBLAS
+    on the same shapes (torch.matmul into a plain [M, N] output, no ReLU, no layout change) is timed
+    beside it for context."""
+    import torch
+
+    import block_causal_linear_relu_b200 as sv
+
+    dev = torch.device("cuda", dev_index)
+    _, tf_burst, tf_sust, _ = peaks()
+    B, N, C, H, D = 2, 10120, 2560, 20, 128
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    x = torch.randn(B, N, C, device=dev, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(3 * H * D, C, device=dev, generator=gen) / C ** 0.5).to(torch.bfloat16)
+    wo = (torch.randn(C, H * D, device=dev, generator=gen) / (H * D) ** 0.5).to(torch.bfloat16)
+    q, k, v = (torch.empty(B, H, N, D, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    y = torch.empty(B, N, C, dtype=torch.bfloat16, device=dev)
+    ws = sv.Workspace(256, dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(dev.index) as clk:
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            e.record(stream)
+            torch.cuda.synchronize()
+        return a.elapsed_time(e) / reps, clk.summary()
+
+    qkv_ms, clk_q = timed(lambda: sv.sv_qkv_projection(x, w, H, D, q=q, k=k, v=v, ws=ws, stream=stream))
+    out_ms, clk_o = timed(lambda: sv.sv_out_projection(v, wo, y=y, ws=ws, stream=stream))
+    x2 = x.view(B * N, C)
+    ref_qkv_ms, _ = timed(lambda: torch.matmul(x2, w.t()))
+    o2 = torch.empty(B * N, H * D, dtype=torch.bfloat16, device=dev)
+    ref_out_ms, _ = timed(lambda: torch.matmul(o2, wo.t()))
+    if ws.status() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout")
+    f_qkv = 2.0 * B * N * C * 3 * H * D
+    f_out = 2.0 * B * N * H * D * C
+    res = {"workload": "SANA-Video 2.0 layer projections: x [2, 10120, 2560] -> q, k, v [2, 20, 10120, 128] (ReLU on "
+                       "q, k); o [2, 20, 10120, 128] -> y [2, 10120, 2560]; bf16, fp32 accumulation",
+           "peak_tflops": tf_burst, "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)"}
+    for name, ms, f, ref_ms, clk in (("qkv", qkv_ms, f_qkv, ref_qkv_ms, clk_q), ("out", out_ms, f_out, ref_out_ms, clk_o)):
+        tf = f / (ms / 1e3) / 1e12
+        res[name] = {"ms": ms, "tflops": tf, "frac": tf / tf_burst, "cublas_ms": ref_ms,
+                     "cublas_tflops": f / (ref_ms / 1e3) / 1e12, "clocks": clk}
+    return res
+
+
 def run_extra(args, name):
     """One configuration alone, as an informational JSON line (not the bench line)."""
     import torch
@@ -582,7 +639,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="leave the other configurations (480p, streaming, 2.0 stack, denoising) out of the line")
-    ap.add_argument("--workload", choices=["720p_prefill", "720p_temporal_conv"] + sorted(EXTRA_WORKLOADS),
+    ap.add_argument("--workload", choices=["720p_prefill", "720p_temporal_conv", "sv2_projections"] + sorted(EXTRA_WORKLOADS),
                     default="720p_prefill",
                     help="the bench line is 720p_prefill; the others print an informational timing line")
     ap.add_argument("--heads", type=int, default=None,
@@ -599,6 +656,12 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload == "sv2_projections":
+        import torch
+        torch.cuda.set_device(0)
+        print(json.dumps({"workload": "sv2_projections", "impl": "ours", **time_proj(max(3, args.steps // 10))}),
+              flush=True)
+        return 0
     if args.workload == "720p_temporal_conv":
         import torch
         torch.cuda.set_device(0)

@@ -24,6 +24,8 @@ from ._native import (  # noqa: F401
     sv_cache_step_noalloc,
     sv_cache_step_noalloc_status,
     sv_linattn_fwd,
+    sv_out_projection,
+    sv_qkv_projection,
     sv_profile_events,
     sv_selftest_wait_timeout,
     sv_temporal_conv,

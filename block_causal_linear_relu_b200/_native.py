@@ -26,7 +26,8 @@ SV_OP_LINATTN_FWD, SV_OP_BLOCK_STATE_UPDATE, SV_OP_BLOCK_CAUSAL_ATTN, SV_OP_CACH
 EXPORTS = (
     "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_workspace_set_mirror", "sv_linattn_fwd",
     "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_cache_step_noalloc",
-    "sv_cache_step_noalloc_status", "sv_temporal_conv", "sv_temporal_conv_step", "sv_profile_events",
+    "sv_cache_step_noalloc_status", "sv_temporal_conv", "sv_temporal_conv_step", "sv_qkv_projection",
+    "sv_out_projection", "sv_profile_events",
     "sv_last_error", "sv_selftest_wait_timeout", "sv_version",
 )
 
@@ -77,6 +78,10 @@ def load() -> ctypes.CDLL:
         lib.sv_temporal_conv.restype = i
         lib.sv_temporal_conv_step.argtypes = [vp, vp, i, i, i, i, vp, vp, vp, i, i, vp]
         lib.sv_temporal_conv_step.restype = i
+        lib.sv_qkv_projection.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]
+        lib.sv_qkv_projection.restype = i
+        lib.sv_out_projection.argtypes = [vp, vp, vp, i, i, i, i, i, vp, sz, vp]
+        lib.sv_out_projection.restype = i
         lib.sv_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
         lib.sv_profile_events.restype = i
         lib.sv_last_error.argtypes = []
@@ -318,4 +323,44 @@ def sv_temporal_conv_step(x, w, carry, commit: bool = True, bias=None, y=None, s
     y = torch.empty_like(x) if y is None else y
     _check(load().sv_temporal_conv_step(_ptr(x), _ptr(y), B, T, S, C, _ptr(w), _ptr(bias), _ptr(carry),
                                         1 if commit else 0, _dt(x), _stream(stream)))
+    return y
+
+
+_proj_ws = {}
+
+
+def _proj_workspace(device, stream):
+    key = (device.index, _stream(stream))
+    ws = _proj_ws.get(key)
+    if ws is None:
+        ws = _proj_ws[key] = Workspace(256, device, stream)
+    ws.check(stream)
+    return ws
+
+
+def sv_qkv_projection(x, w_qkv, H: int, D: int, q=None, k=None, v=None, ws: Workspace | None = None, stream=None):
+    """x [B, N, C] bf16, w_qkv [3*H*D, C] bf16 -> (ReLU(q), ReLU(k), v), each [B, H, N, D] bf16."""
+    if not x.is_cuda or x.dim() != 3 or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bfloat16 CUDA tensor [B, N, C]")
+    B, N, C = x.shape
+    if tuple(w_qkv.shape) != (3 * H * D, C) or w_qkv.dtype != torch.bfloat16 or not w_qkv.is_contiguous():
+        raise ValueError("w_qkv must be a contiguous bfloat16 [3*H*D, C] tensor")
+    q, k, v = (torch.empty(B, H, N, D, dtype=torch.bfloat16, device=x.device) if t is None else t for t in (q, k, v))
+    ws = ws if ws is not None else _proj_workspace(x.device, stream)
+    _check(load().sv_qkv_projection(_ptr(x), _ptr(w_qkv), _ptr(q), _ptr(k), _ptr(v), B, N, C, H, D, ws.ptr, ws.nbytes,
+                                    _stream(stream)))
+    return q, k, v
+
+
+def sv_out_projection(o, w_o, y=None, ws: Workspace | None = None, stream=None):
+    """o [B, H, N, D] bf16, w_o [C_out, H*D] bf16 -> y [B, N, C_out] bf16."""
+    if not o.is_cuda or o.dim() != 4 or o.dtype != torch.bfloat16 or not o.is_contiguous():
+        raise ValueError("o must be a contiguous bfloat16 CUDA tensor [B, H, N, D]")
+    B, H, N, D = o.shape
+    if w_o.dim() != 2 or w_o.shape[1] != H * D or w_o.dtype != torch.bfloat16 or not w_o.is_contiguous():
+        raise ValueError("w_o must be a contiguous bfloat16 [C_out, H*D] tensor")
+    C_out = w_o.shape[0]
+    y = torch.empty(B, N, C_out, dtype=torch.bfloat16, device=o.device) if y is None else y
+    ws = ws if ws is not None else _proj_workspace(o.device, stream)
+    _check(load().sv_out_projection(_ptr(o), _ptr(w_o), _ptr(y), B, N, H, D, C_out, ws.ptr, ws.nbytes, _stream(stream)))
     return y

@@ -12,7 +12,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsvlinattn.so")
-SOURCES = ["sv_kernels.cu", "sv_api.cu", "sv_noalloc.cu", "sv_selftest.cu", "sv_conv.cu"]
+SOURCES = ["sv_kernels.cu", "sv_api.cu", "sv_noalloc.cu", "sv_selftest.cu", "sv_conv.cu", "sv_proj.cu"]
 HEADERS = ["sv_ptx.cuh", "sv_geometry.h", "sv_internal.h"]
 
 NVCC_FLAGS = [

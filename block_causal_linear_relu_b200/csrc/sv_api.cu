@@ -145,6 +145,27 @@ sv_status encode_map_uncached(CUtensorMap* m, const void* base, uint64_t rows, u
   return SV_OK;
 }
 
+}  // namespace
+
+namespace sv {
+sv_status encode_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                         const uint32_t box[4]) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(SV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t st[3] = {strides[0], strides[1], strides[2]};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, st, bx, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SV_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return SV_OK;
+}
+}  // namespace sv
+
+namespace {
+
 // [BH, N, D] bf16 seen as [BH, nblk, L, D] blocks; the shorter last block gets its own map so that
 // TMA bounds-checks every tile against its own block (zero fill on loads, clipping on stores).
 sv_status make_block_maps(sv::BlockMaps& bm, const void* x, const Geom& g, uint32_t box_rows) {

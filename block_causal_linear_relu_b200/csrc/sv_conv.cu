@@ -82,14 +82,35 @@ __global__ void __launch_bounds__(kConvThreads) temporal_conv_kernel(const T* x,
   const int c0 = static_cast<int>(col - bs * per_row) * NV;
   const int b = static_cast<int>(bs / S);
   const int s = static_cast<int>(bs - static_cast<long long>(b) * S);
-  float w0[NV], w1[NV], w2[NV], bb[NV];
+  // the group's 3 * NV taps are contiguous (16-byte aligned: NV * 12 bytes per group), as are its NV
+  // biases: vector loads
+  float wt[3 * NV], w0[NV], w1[NV], w2[NV], bb[NV];
+#pragma unroll
+  for (int i = 0; i < 3 * NV / 4; ++i) {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(w + c0 * 3) + i);
+    wt[4 * i] = f.x;
+    wt[4 * i + 1] = f.y;
+    wt[4 * i + 2] = f.z;
+    wt[4 * i + 3] = f.w;
+  }
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
-    w0[i] = __ldg(w + (c0 + i) * 3);
-    w1[i] = __ldg(w + (c0 + i) * 3 + 1);
-    w2[i] = __ldg(w + (c0 + i) * 3 + 2);
-    bb[i] = bias != nullptr ? __ldg(bias + c0 + i) : 0.f;
+    w0[i] = wt[3 * i];
+    w1[i] = wt[3 * i + 1];
+    w2[i] = wt[3 * i + 2];
   }
+#pragma unroll
+  for (int i = 0; i < NV / 4; ++i) {
+    const float4 f = bias != nullptr ? __ldg(reinterpret_cast<const float4*>(bias + c0) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    bb[4 * i] = f.x;
+    bb[4 * i + 1] = f.y;
+    bb[4 * i + 2] = f.z;
+    bb[4 * i + 3] = f.w;
+  }
+  // x (or the carry) may come from the previous kernel in the stream: wait for it here, after the
+  // weights, so that the launch overlaps the previous kernel's tail
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const size_t frame = static_cast<size_t>(S) * C;
   const size_t base = (static_cast<size_t>(b) * Tf * S + s) * C + c0;
   const T* xp = x + base;
@@ -150,19 +171,30 @@ sv_status run_conv(const void* x, void* y, int B, int T, int S, int C, int L, co
   const auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
   if (!al(x, 16) || !al(y, 16) || (carry != nullptr && !al(carry, 16)))
     return conv_fail(SV_ERR_INVALID_ARG, "x, y and carry must be 16-byte aligned");
-  if (!al(w, 4) || (bias != nullptr && !al(bias, 4))) return conv_fail(SV_ERR_INVALID_ARG, "w or bias misaligned");
+  if (!al(w, 16) || (bias != nullptr && !al(bias, 16)))
+    return conv_fail(SV_ERR_INVALID_ARG, "w and bias must be 16-byte aligned");
   const long long ncols = static_cast<long long>(B) * S * (C / nv);
   const long long nblocks = (ncols + kConvThreads - 1) / kConvThreads;
   if (nblocks > 0x7fffffffLL) return conv_fail(SV_ERR_UNSUPPORTED, "too many columns");
+  // programmatic dependent launch: the CTAs may start while the previous kernel drains; they wait
+  // (griddepcontrol.wait) before touching x, y or the carry
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nblocks));
+  cfg.blockDim = dim3(kConvThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (dt == SV_BF16)
-    temporal_conv_kernel<__nv_bfloat16><<<static_cast<unsigned>(nblocks), kConvThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), B, T, S, C, L, w, bias,
-        static_cast<__nv_bfloat16*>(carry), commit, ncols);
+    e = cudaLaunchKernelEx(&cfg, temporal_conv_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x),
+                           static_cast<__nv_bfloat16*>(y), B, T, S, C, L, w, bias, static_cast<__nv_bfloat16*>(carry),
+                           commit, ncols);
   else
-    temporal_conv_kernel<float><<<static_cast<unsigned>(nblocks), kConvThreads, 0, stream>>>(
-        static_cast<const float*>(x), static_cast<float*>(y), B, T, S, C, L, w, bias, static_cast<float*>(carry),
-        commit, ncols);
-  const cudaError_t e = cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, temporal_conv_kernel<float>, static_cast<const float*>(x), static_cast<float*>(y), B,
+                           T, S, C, L, w, bias, static_cast<float*>(carry), commit, ncols);
   if (e != cudaSuccess) {
     snprintf(msg, sizeof(msg), "temporal conv launch: %s", cudaGetErrorString(e));
     return conv_fail(SV_ERR_CUDA, msg);

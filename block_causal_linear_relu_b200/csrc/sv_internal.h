@@ -60,6 +60,10 @@ cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g
                         float* S_out, float* z_out, void* ptiles_bf16, float* p32, uint32_t* out_chunks,
                         cudaStream_t st);
 
+// A 4-D bf16 tensor map with 128-byte swizzle (dims innermost first, byte strides of dims 1..3).
+sv_status encode_bf16_4d(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides[3],
+                         const uint32_t box[4]);
+
 // Records `msg` as the calling thread's sv_last_error() text and returns `status`.
 sv_status set_last_error(sv_status status, const char* msg);
 

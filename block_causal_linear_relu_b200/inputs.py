@@ -74,3 +74,14 @@ def draw_conv(shape, seed: int, dtype: str = BF16):
     w = (rng.standard_normal((C, 3), dtype=np.float32) * np.float32(0.5)).astype(np.float32)
     b = (rng.standard_normal((C,), dtype=np.float32) * np.float32(0.5)).astype(np.float32)
     return (f32_to_bf16_bits(x) if dtype == BF16 else x), w, b
+
+
+def draw_proj(x_shape, n_out: int, seed: int):
+    """Inputs of a projection: x ~ N(0, 1) of `x_shape` (last dim = input features C), then the
+    weight [n_out, C] ~ N(0, 1/C) (synthetic: the pages give no trained weights), from one seeded
+    generator in that order; both as bf16 bit patterns (round to nearest even)."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(x_shape, dtype=np.float32)
+    C = x_shape[-1]
+    w = (rng.standard_normal((n_out, C), dtype=np.float32) * np.float32(1.0 / np.sqrt(C))).astype(np.float32)
+    return f32_to_bf16_bits(x), f32_to_bf16_bits(w)

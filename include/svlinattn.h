@@ -176,7 +176,8 @@ sv_status sv_cache_step_noalloc_status(sv_stream_t stream, uint32_t* code);
  * blk(t) = floor(t / frames_per_block), x[-1] = 0; the last block may be shorter.
  * x, y: DEVICE pointers to contiguous [B, T, S, C] tensors (T latent frames of S tokens, C channels,
  * C fastest), element type dt, 16-byte aligned; C a multiple of 8 (bf16) or 4 (fp32). y may equal x.
- * w: DEVICE fp32 [C][3]; bias: DEVICE fp32 [C] or NULL. Computed in fp32, rounded once to dt. */
+ * w: DEVICE fp32 [C][3]; bias: DEVICE fp32 [C] or NULL; both 16-byte aligned. Computed in fp32,
+ * rounded once to dt. */
 sv_status sv_temporal_conv(const void* x, void* y, int B, int T, int S, int C, int frames_per_block, const float* w,
                            const float* bias, sv_dtype dt, sv_stream_t stream);
 
@@ -188,6 +189,27 @@ sv_status sv_temporal_conv(const void* x, void* y, int B, int T, int S, int C, i
  * the whole sequence (talk, causal FFN with temporal conv passage). */
 sv_status sv_temporal_conv_step(const void* x, void* y, int B, int T, int S, int C, const float* w, const float* bias,
                                 void* carry, int commit, sv_dtype dt, sv_stream_t stream);
+
+/* The Q/K/V projection of a linear-attention layer with the feature map in its epilogue (SANA-Video
+ * model-family page, 2.0 paragraph: hidden size 2560 = 20 heads x 128 features; the ReLU feature
+ * map of the library's operation). The pages print no formula; this library's reading is a bias-free
+ * linear map with one fused weight:
+ *     [q | k | v] = x W_qkv^T,   q = ReLU(.),  k = ReLU(.),  v linear,
+ * W_qkv [3*H*D, C] row-major bf16 (row f = output feature f: Q features 0..H*D-1, then K, then V;
+ * head h owns features h*D .. h*D+D-1 of each). x: [B, N, C] bf16; q, k, v: [B, H, N, D] bf16 (the
+ * layout the attention calls read; ReLU applied again there changes nothing). fp32 accumulation,
+ * one bf16 rounding. All pointers are DEVICE pointers, 16-byte aligned. Supported: D = 64 or 128,
+ * C a multiple of 64. ws: a workspace of at least 256 bytes (sv_workspace_init) whose status word
+ * reports a device-side timeout (sv_device_status). */
+sv_status sv_qkv_projection(const void* x, const void* w_qkv, void* q, void* k, void* v, int B, int N, int C, int H,
+                            int D, void* ws, size_t ws_bytes, sv_stream_t stream);
+
+/* The output projection after the attention (same page and reading): y = o_cat W_o^T with the
+ * heads of o [B, H, N, D] concatenated feature-major (o_cat[b, n, h*D + d] = o[b, h, n, d], read in
+ * place, no copy), W_o [C_out, H*D] row-major bf16, y [B, N, C_out] bf16. D = 64 or 128, C_out a
+ * multiple of 64; ws as for sv_qkv_projection. */
+sv_status sv_out_projection(const void* o, const void* w_o, void* y, int B, int N, int H, int D, int C_out, void* ws,
+                            size_t ws_bytes, sv_stream_t stream);
 
 /* Optional timing hook for benchmarks. With events != NULL (n == 4 cudaEvent_t handles owned by
  * the caller), the calling thread's following forward calls (sv_linattn_fwd, sv_block_causal_attn,
