@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kConvThreads) temporal_conv_kernel(const T* x,
   const int s = static_cast<int>(bs - static_cast<long long>(b) * S);
   // the group's 3 * NV taps are contiguous (16-byte aligned: NV * 12 bytes per group), as are its NV
   // biases: vector loads
-  float wt[3 * NV], w0[NV], w1[NV], w2[NV], bb[NV];
+  float wt[3 * NV], bb[NV];  // wt[3 i + j]: tap j (t - 1, t, t + 1) of channel c0 + i
 #pragma unroll
   for (int i = 0; i < 3 * NV / 4; ++i) {
     const float4 f = __ldg(reinterpret_cast<const float4*>(w + c0 * 3) + i);
@@ -92,12 +92,6 @@ __global__ void __launch_bounds__(kConvThreads) temporal_conv_kernel(const T* x,
     wt[4 * i + 1] = f.y;
     wt[4 * i + 2] = f.z;
     wt[4 * i + 3] = f.w;
-  }
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    w0[i] = wt[3 * i];
-    w1[i] = wt[3 * i + 1];
-    w2[i] = wt[3 * i + 2];
   }
 #pragma unroll
   for (int i = 0; i < NV / 4; ++i) {
@@ -140,9 +134,9 @@ __global__ void __launch_bounds__(kConvThreads) temporal_conv_kernel(const T* x,
       const bool same = t + 1 < Tf && (t + 1) / L == t / L;  // the right neighbour is in t's block
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
-        float a = fmaf(w0[i], prev[i], bb[i]);
-        a = fmaf(w1[i], cur[i], a);
-        out[i] = same ? fmaf(w2[i], nxt[i], a) : a;
+        float a = fmaf(wt[3 * i], prev[i], bb[i]);
+        a = fmaf(wt[3 * i + 1], cur[i], a);
+        out[i] = same ? fmaf(wt[3 * i + 2], nxt[i], a) : a;
         prev[i] = cur[i];
         cur[i] = nxt[i];
       }

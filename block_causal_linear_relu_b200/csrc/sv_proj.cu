@@ -11,7 +11,11 @@
 // 2-5 drain TMEM in 64-column chunks: ReLU where the chunk belongs to Q or K, bf16, a swizzled
 // staging buffer, and a TMA store of 32 rows x 64 features into the chunk's tensor, head and
 // features. Rows are tiled per batch (a tile never holds two batches' tokens); the last row tile of
-// a batch is zero-filled on load and clipped on store by the tensor maps.
+// a batch is zero-filled on load and clipped on store by the tensor maps. Tiles are numbered column
+// tile fastest, so the CTAs working at any moment share a few row tiles of A (read from DRAM once)
+// and sweep the whole weight, which stays in L2 (39 MB for the fused Q/K/V weight at hidden 2560);
+// numbered the other way, every column tile streamed all of A through L2 again (measured: 3.15 GB of
+// DRAM reads for 143 MB of operands).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < g.tiles && ok; tile += gridDim.x) {
-        const int m = tile % g.mt, n = tile / g.mt;
+        const int n = tile % g.nt, m = tile / g.nt;
         const int b = m / g.mtb, i0 = (m - b * g.mtb) * kBM, n0 = n * kBN;
         for (int kc = 0; kc < g.kchunks; ++kc, ++it) {
           const int s = it % kPStages;
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int a = tl & 1;
       if (!all_lanes(mbar_wait(&accf[a], (tl >> 1) & 1, status, 0x5400u | a))) break;
       tc_fence_after();
-      const int m = tile % g.mt, n = tile / g.mt;
+      const int n = tile % g.nt, m = tile / g.nt;
       const int b = m / g.mtb, i0 = (m - b * g.mtb) * kBM;
       const int row0 = i0 + q * 32;  // first token of this warp's slice
       const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * kBN);
