@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <mutex>
 
 #include "../../include/svlinattn.h"
 #include "sv_internal.h"
@@ -241,15 +242,30 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
+// The kernels' shared-memory attribute, set once per device (and per kernel), thread-safe.
+template <bool kQKV>
+cudaError_t ensure_attr() {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static bool done[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(proj_kernel<kQKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
+}
+
 template <bool kQKV>
 cudaError_t launch_proj(const CUtensorMap& a, const CUtensorMap& bm, const CUtensorMap& o0, const CUtensorMap& o1,
                         const CUtensorMap& o2, const PGeom& g, uint32_t* status, int sm_count, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(proj_kernel<kQKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const cudaError_t ea = ensure_attr<kQKV>();
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(g.tiles < sm_count ? g.tiles : sm_count));
   cfg.blockDim = dim3(kPThreads);

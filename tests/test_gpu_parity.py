@@ -102,7 +102,9 @@ def test_fp32_shapes(sv, B, H, N, D, L):
     (2, 1, 300, 8, 77),        # D = 8: a 16-byte row
     (1, 2, 400, 72, 150),      # D = 72 (second atom holds 8 features)
     (1, 1, 260, 120, 260),     # D = 120, bidirectional
-    (2, 40, 500, 16, 500),     # one block per head, 80 heads: the flag-synchronised kernel, D = 16
+    (2, 40, 500, 16, 500),     # one block per head, 80 heads: the one-launch kernel, D = 16
+    (4, 100, 100, 64, 100),    # 400 one-tile heads: CTAs span three heads, the one-launch kernel's
+                               # flag-and-slot exchange (no L2 accumulators)
 ])
 def test_bf16_shapes(sv, B, H, N, D, L):
     st, (q, k, v) = inputs((B, H, N, D), 1, "bf16")
