@@ -19,3 +19,11 @@ from .linattn import (  # noqa: F401
 )
 from .projection import out_projection, qkv_projection  # noqa: F401,E402
 from .temporal_conv import centred_conv, temporal_conv_block_causal, temporal_conv_step  # noqa: F401,E402
+from .rope import (  # noqa: F401,E402
+    block_causal_attn_rope,
+    bruteforce_rope,
+    default_pairs,
+    rope3d_angles,
+    rotate_pairs,
+    token_positions,
+)
