@@ -13,12 +13,15 @@ from ._native import (  # noqa: F401
     SV_OP_BLOCK_STATE_UPDATE,
     SV_OP_CACHE_STEP,
     SV_OP_LINATTN_FWD,
+    Rope3dTable,
     SvError,
+    SvRope3d,
     Workspace,
     lib_path,
     load,
     make_workspace,
     sv_block_causal_attn,
+    sv_block_causal_attn_rope,
     sv_block_state_update,
     sv_cache_step,
     sv_cache_step_noalloc,
@@ -27,6 +30,8 @@ from ._native import (  # noqa: F401
     sv_out_projection,
     sv_qkv_projection,
     sv_profile_events,
+    sv_rope3d_table,
+    sv_rope3d_table_bytes,
     sv_selftest_wait_timeout,
     sv_temporal_conv,
     sv_temporal_conv_step,

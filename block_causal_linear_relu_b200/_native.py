@@ -27,9 +27,17 @@ EXPORTS = (
     "sv_workspace_bytes", "sv_workspace_init", "sv_device_status", "sv_workspace_set_mirror", "sv_linattn_fwd",
     "sv_block_state_update", "sv_block_causal_attn", "sv_cache_step", "sv_cache_step_noalloc",
     "sv_cache_step_noalloc_status", "sv_temporal_conv", "sv_temporal_conv_step", "sv_qkv_projection",
-    "sv_out_projection", "sv_profile_events",
+    "sv_out_projection", "sv_rope3d_table_bytes", "sv_rope3d_table", "sv_block_causal_attn_rope", "sv_profile_events",
     "sv_last_error", "sv_selftest_wait_timeout", "sv_version",
 )
+
+
+class SvRope3d(ctypes.Structure):
+    """The C descriptor sv_rope3d (include/svlinattn.h)."""
+
+    _fields_ = [("table", ctypes.c_void_p), ("frames", ctypes.c_int), ("height", ctypes.c_int),
+                ("width", ctypes.c_int), ("D", ctypes.c_int), ("pairs_t", ctypes.c_int), ("pairs_h", ctypes.c_int),
+                ("pairs_w", ctypes.c_int), ("frame0", ctypes.c_int)]
 
 
 class SvError(RuntimeError):
@@ -82,6 +90,13 @@ def load() -> ctypes.CDLL:
         lib.sv_qkv_projection.restype = i
         lib.sv_out_projection.argtypes = [vp, vp, vp, i, i, i, i, i, vp, sz, vp]
         lib.sv_out_projection.restype = i
+        lib.sv_rope3d_table_bytes.argtypes = [i, i, i, i]
+        lib.sv_rope3d_table_bytes.restype = sz
+        lib.sv_rope3d_table.argtypes = [vp, sz, i, i, i, i, i, i, i, f, vp]
+        lib.sv_rope3d_table.restype = i
+        lib.sv_block_causal_attn_rope.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp, vp,
+                                                  ctypes.POINTER(SvRope3d), vp, sz, vp]
+        lib.sv_block_causal_attn_rope.restype = i
         lib.sv_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i]
         lib.sv_profile_events.restype = i
         lib.sv_last_error.argtypes = []
@@ -364,3 +379,51 @@ def sv_out_projection(o, w_o, y=None, ws: Workspace | None = None, stream=None):
     ws = ws if ws is not None else _proj_workspace(o.device, stream)
     _check(load().sv_out_projection(_ptr(o), _ptr(w_o), _ptr(y), B, N, H, D, C_out, ws.ptr, ws.nbytes, _stream(stream)))
     return y
+
+
+def sv_rope3d_table_bytes(frames: int, height: int, width: int, D: int) -> int:
+    n = load().sv_rope3d_table_bytes(frames, height, width, D)
+    if n == 0:
+        raise SvError(SV_ERR_INVALID_ARG, load().sv_last_error().decode())
+    return n
+
+
+class Rope3dTable:
+    """The device (cos, sin) table of the 3D rotary embedding for one grid and feature split, built
+    by sv_rope3d_table; `desc(frame0)` gives the sv_rope3d descriptor of a call."""
+
+    def __init__(self, frames: int, height: int, width: int, D: int, pairs, base: float = 10000.0, device=None,
+                 stream=None):
+        pt, ph, pw = (int(p) for p in pairs)
+        nbytes = sv_rope3d_table_bytes(frames, height, width, D)
+        self.table = torch.empty(nbytes // 4, dtype=torch.float32, device=device or torch.device("cuda"))
+        self.frames, self.height, self.width, self.D, self.pairs = frames, height, width, D, (pt, ph, pw)
+        _check(load().sv_rope3d_table(self.table.data_ptr(), nbytes, frames, height, width, D, pt, ph, pw, base,
+                                      _stream(stream)))
+
+    def desc(self, frame0: int = 0) -> SvRope3d:
+        pt, ph, pw = self.pairs
+        return SvRope3d(self.table.data_ptr(), self.frames, self.height, self.width, self.D, pt, ph, pw, int(frame0))
+
+
+def sv_rope3d_table(frames: int, height: int, width: int, D: int, pairs, base: float = 10000.0, device=None,
+                    stream=None) -> Rope3dTable:
+    return Rope3dTable(frames, height, width, D, pairs, base, device, stream)
+
+
+def sv_block_causal_attn_rope(q, k, v, block_len: int, rope: Rope3dTable, frame0: int = 0, o=None, eps: float = 1e-6,
+                              S_in=None, z_in=None, S_out=None, z_out=None, ws: Workspace | None = None, stream=None):
+    """sv_block_causal_attn with the 3D rotary embedding of the numerator; returns o."""
+    o = torch.empty_like(q) if o is None else o
+    B, H, N, D = _qkv(q, k, v, o)
+    for t in (S_in, z_in, S_out, z_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or t.device != q.device):
+            raise ValueError("S/z must be contiguous float32 tensors on q's device")
+    if rope.table.device != q.device:
+        raise ValueError("the rope table must live on q's device")
+    ws = _ws(ws, SV_OP_BLOCK_CAUSAL_ATTN, q, block_len, stream)
+    d = rope.desc(frame0)
+    _check(load().sv_block_causal_attn_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, D, int(block_len), _dt(q),
+                                            eps, _ptr(S_in), _ptr(z_in), _ptr(S_out), _ptr(z_out), ctypes.byref(d),
+                                            ws.ptr, ws.nbytes, _stream(stream)))
+    return o

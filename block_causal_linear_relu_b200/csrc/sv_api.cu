@@ -260,9 +260,10 @@ sv_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   } while (0)
 
 // The whole forward path: state reduction -> partial combine + prefix -> output GEMM.
+// With `rope` (the rotary form) the bf16 work always takes the three-kernel path.
 sv_status run_forward(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D, int L,
                       sv_dtype dt, float eps, const float* S_in, const float* z_in, float* S_out, float* z_out,
-                      void* ws, size_t ws_bytes, cudaStream_t stream) {
+                      void* ws, size_t ws_bytes, cudaStream_t stream, const sv::RopeDev* rope = nullptr) {
   SV_TRY(check_sizes(B, H, N, D, L, dt));
   SV_TRY(check_io("q", q));
   SV_TRY(check_io("k", k));
@@ -289,7 +290,7 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
   cudaError_t e;
   if (dt == SV_BF16) {
     // one block per head and few heads: one thread-block cluster per head (a single launch)
-    const int C = g.nblk == 1 ? sv::cluster_size(g, di.sm_count) : 0;
+    const int C = g.nblk == 1 && rope == nullptr ? sv::cluster_size(g, di.sm_count) : 0;
     if (C > 0) {
       sv::ClusterMaps cm;
       SV_TRY(encode_map(&cm.k, k, g.N, 1, g, sv::kTile));
@@ -316,7 +317,7 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
     SV_TRY(make_block_maps(mv, v, g, sv::kTile));
     SV_TRY(make_block_maps(mq, q, g, sv::kTile));
     SV_TRY(make_block_maps(mo, o, g, 32));
-    if (g.nblk == 1) {  // one block per head, many heads: a single launch of co-resident CTAs
+    if (g.nblk == 1 && rope == nullptr) {  // one block per head, many heads: a single launch of co-resident CTAs
       prof_mark(0, stream);
       e = sv::launch_fused_bf16(mk, mv, mq, mo, g, partials, segcta, flags, pre, S_in, z_in, S_out, z_out, eps,
                                 status, stream);
@@ -327,29 +328,71 @@ sv_status run_forward(const void* q, const void* k, const void* v, void* o, int 
       return SV_OK;
     }
     prof_mark(0, stream);
-    e = sv::launch_state_bf16(mk, mv, g, partials, segcta, status, stream);
+    e = sv::launch_state_bf16(mk, mv, g, partials, segcta, status, stream, rope);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
     prof_mark(1, stream);
     e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, pre, nullptr, status + 6, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     prof_mark(2, stream);
-    e = sv::launch_out_bf16(mq, mo, g, pre, eps, status, stream);
+    e = sv::launch_out_bf16(mq, mo, g, pre, eps, status, stream, rope);
     if (e != cudaSuccess) return cuda_fail(e, "output kernel launch");
     prof_mark(3, stream);
   } else {
     float* p32 = static_cast<float*>(pre);
     prof_mark(0, stream);
     e = sv::launch_state_f32(static_cast<const float*>(k), static_cast<const float*>(v), g, partials, segcta,
-                             status, stream);
+                             status, stream, rope);
     if (e != cudaSuccess) return cuda_fail(e, "state kernel launch");
     prof_mark(1, stream);
     e = sv::launch_scan(partials, segcta, g, S_in, z_in, S_out, z_out, nullptr, p32, status + 6, stream);
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     prof_mark(2, stream);
-    e = sv::launch_out_f32(static_cast<const float*>(q), static_cast<float*>(o), g, p32, eps, status, stream);
+    e = sv::launch_out_f32(static_cast<const float*>(q), static_cast<float*>(o), g, p32, eps, status, stream, rope);
     if (e != cudaSuccess) return cuda_fail(e, "output kernel launch");
     prof_mark(3, stream);
   }
+  return SV_OK;
+}
+
+// Table size check shared by sv_rope3d_table_bytes and the attention call: the grid and D.
+sv_status check_rope_grid(int frames, int height, int width, int D) {
+  if (frames < 1 || height < 1 || width < 1)
+    return fail(SV_ERR_INVALID_ARG, "rope grid frames=%d height=%d width=%d must all be >= 1", frames, height, width);
+  if (D < 2 || D > 128 || D % 2 != 0) return fail(SV_ERR_INVALID_ARG, "rope D=%d must be even, in [2, 128]", D);
+  if (static_cast<long long>(frames) + height + width > (1ll << 24))
+    return fail(SV_ERR_INVALID_ARG, "rope table of %lld rows is too large",
+                static_cast<long long>(frames) + height + width);
+  if (static_cast<long long>(height) * width > 0x7fffffffll)
+    return fail(SV_ERR_INVALID_ARG, "rope grid height*width overflows int");
+  return SV_OK;
+}
+
+sv_status check_rope_pairs(int D, int pt, int ph, int pw) {
+  if (pt < 0 || ph < 0 || pw < 0 || 2 * (static_cast<long long>(pt) + ph + pw) != D)
+    return fail(SV_ERR_INVALID_ARG, "rope pairs (%d, %d, %d) must be >= 0 and sum to D/2 = %d", pt, ph, pw, D / 2);
+  return SV_OK;
+}
+
+// Checks a descriptor against the call's N and D and turns it into the kernels' form.
+sv_status rope_for(sv::RopeDev& rd, const sv_rope3d* r, int N, int D) {
+  if (r == nullptr) return fail(SV_ERR_INVALID_ARG, "rope descriptor is NULL");
+  SV_TRY(check_rope_grid(r->frames, r->height, r->width, r->D));
+  SV_TRY(check_rope_pairs(r->D, r->pairs_t, r->pairs_h, r->pairs_w));
+  if (r->D != D) return fail(SV_ERR_INVALID_ARG, "rope table D=%d differs from the call's D=%d", r->D, D);
+  if (r->table == nullptr || !aligned(r->table, 16)) return fail(SV_ERR_INVALID_ARG, "rope table is NULL or not 16-byte aligned");
+  const long long hw = static_cast<long long>(r->height) * r->width;
+  if (r->frame0 < 0 || r->frame0 + (static_cast<long long>(N) - 1) / hw >= r->frames)
+    return fail(SV_ERR_INVALID_ARG, "rope frame0=%d with N=%d tokens of %lld per frame leaves the table's %d frames",
+                r->frame0, N, hw, r->frames);
+  rd.tab = reinterpret_cast<const float2*>(r->table);
+  rd.half = D / 2;
+  rd.hw = static_cast<int>(hw);
+  rd.w = r->width;
+  rd.f0 = r->frame0;
+  rd.row_h = r->frames;
+  rd.row_w = r->frames + r->height;
+  rd.pt = r->pairs_t;
+  rd.pth = r->pairs_t + r->pairs_h;
   return SV_OK;
 }
 
@@ -447,6 +490,39 @@ sv_status sv_cache_step(const void* q, const void* k, const void* v, void* o, in
   SV_TRY(check_cache("z", z, true));
   return run_forward(q, k, v, o, B, H, N, D, N, dt, eps, S, z, commit ? S : nullptr, commit ? z : nullptr, ws,
                      ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t sv_rope3d_table_bytes(int frames, int height, int width, int D) {
+  if (check_rope_grid(frames, height, width, D) != SV_OK) return 0;
+  return (static_cast<size_t>(frames) + height + width) * static_cast<size_t>(D / 2) * 8;
+}
+
+sv_status sv_rope3d_table(float* table, size_t table_bytes, int frames, int height, int width, int D, int pairs_t,
+                          int pairs_h, int pairs_w, float base, sv_stream_t stream) {
+  SV_TRY(check_rope_grid(frames, height, width, D));
+  SV_TRY(check_rope_pairs(D, pairs_t, pairs_h, pairs_w));
+  if (!std::isfinite(base) || base <= 1.f) return fail(SV_ERR_INVALID_ARG, "rope base must be finite and > 1");
+  if (table == nullptr || !aligned(table, 16)) return fail(SV_ERR_INVALID_ARG, "table is NULL or not 16-byte aligned");
+  const size_t need = sv_rope3d_table_bytes(frames, height, width, D);
+  if (table_bytes < need) return fail(SV_ERR_INVALID_ARG, "table_bytes=%zu < %zu", table_bytes, need);
+  DevInfo di;
+  SV_TRY(device_info(di, false));
+  const cudaError_t e = sv::launch_rope_table(reinterpret_cast<float2*>(table), frames, height, width, D / 2, pairs_t,
+                                              pairs_h, pairs_w, static_cast<double>(base),
+                                              reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rope table kernel launch");
+  return SV_OK;
+}
+
+sv_status sv_block_causal_attn_rope(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                                    int block_len, sv_dtype dt, float eps, const float* S_in, const float* z_in,
+                                    float* S_out, float* z_out, const sv_rope3d* rope, void* ws, size_t ws_bytes,
+                                    sv_stream_t stream) {
+  SV_TRY(check_sizes(B, H, N, D, block_len, dt));
+  sv::RopeDev rd;
+  SV_TRY(rope_for(rd, rope, N, D));
+  return run_forward(q, k, v, o, B, H, N, D, block_len, dt, eps, S_in, z_in, S_out, z_out, ws, ws_bytes,
+                     reinterpret_cast<cudaStream_t>(stream), &rd);
 }
 
 sv_status sv_block_state_update(const void* k, const void* v, int B, int H, int N, int D, sv_dtype dt, float* S,

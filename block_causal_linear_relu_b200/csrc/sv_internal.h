@@ -27,11 +27,24 @@ struct BlockMaps {
   CUtensorMap last;
 };
 
-// bf16 path
+// 3D rotary embedding of the feature-mapped q and k, applied to the numerator only
+// (sv_block_causal_attn_rope). tab holds (cos, sin) per (row, pair): rows [0, row_h) are frame
+// positions, [row_h, row_w) grid rows, [row_w, ...) grid columns; `half` = D / 2 pairs per row.
+// Token n of a (batch, head) sequence sits at frame f0 + n / hw, row (n % hw) / w, column n % w.
+// Pairs [0, pt) turn with the frame, [pt, pth) with the row, [pth, half) with the column.
+struct RopeDev {
+  const float2* tab;
+  int half, hw, w, f0, row_h, row_w, pt, pth;
+};
+
+// bf16 path (rope: nullptr, or the rotation of the numerator's features)
 cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,
-                              uint32_t* status, cudaStream_t st);
+                              uint32_t* status, cudaStream_t st, const RopeDev* rope = nullptr);
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles,
-                            float eps, uint32_t* status, cudaStream_t st);
+                            float eps, uint32_t* status, cudaStream_t st, const RopeDev* rope = nullptr);
+// fills a RopeDev table: rows = frames + height + width, `half` pairs per row
+cudaError_t launch_rope_table(float2* tab, int frames, int height, int width, int half, int pt, int ph, int pw,
+                              double base, cudaStream_t st);
 // bf16, whole sequence in one block: state -> combine -> output in one cooperative launch
 cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
                               const Geom& g, float* partials, int2* segcta, uint64_t* flags, void* ptiles,
@@ -51,9 +64,9 @@ cudaError_t launch_cluster_bf16(const ClusterMaps& m, const Geom& g, int C, floa
                                 cudaStream_t st);
 // fp32 path
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
-                             uint32_t* status, cudaStream_t st);
+                             uint32_t* status, cudaStream_t st, const RopeDev* rope = nullptr);
 cudaError_t launch_out_f32(const float* q, float* o, const Geom& g, const float* p32, float eps,
-                           uint32_t* status, cudaStream_t st);
+                           uint32_t* status, cudaStream_t st, const RopeDev* rope = nullptr);
 // both paths: combine partials, inclusive prefix over blocks, optional final cache
 // out_chunks: the output kernel's dynamic-chunk counter (workspace header bytes 24..27), reset here.
 cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g, const float* S_in, const float* z_in,

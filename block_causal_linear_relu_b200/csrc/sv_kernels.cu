@@ -20,6 +20,10 @@
 // the state roles, a per-head combine shared by the CTAs that cover the head, synchronised through
 // release/acquire flags, then the output roles).
 // The fp32 I/O path runs the same three steps with SIMT fp32 kernels.
+// With the 3D rotary embedding (sv_block_causal_attn_rope) the three-kernel path turns the
+// feature-mapped K and Q tiles in shared memory after the MMAs that need them unturned (the z
+// column of the state, the denominator of the output) have read them, and before the MMAs of the
+// numerator: the ReLU warps run one tile behind with the turn.
 #include <cuda_bf16.h>
 
 #include <cstdlib>
@@ -57,6 +61,57 @@ __device__ __forceinline__ void relu_tile_inplace(uint8_t* tile, int nchunks, in
     x.z = relu_bf16x2(x.z);
     x.w = relu_bf16x2(x.w);
     p[i] = x;
+  }
+}
+
+// ---- 3D rotary embedding of the feature-mapped features (numerator of the rotated form) ----
+// Table rows of token n's frame, grid row and grid column.
+__device__ __forceinline__ void rope_rows(const RopeDev& rp, int n, const float2*& rt, const float2*& rh,
+                                          const float2*& rw) {
+  const int f = n / rp.hw;
+  const int rem = n - f * rp.hw;
+  const int y = rem / rp.w;
+  const int x = rem - y * rp.w;
+  rt = rp.tab + static_cast<size_t>(rp.f0 + f) * rp.half;
+  rh = rp.tab + static_cast<size_t>(rp.row_h + y) * rp.half;
+  rw = rp.tab + static_cast<size_t>(rp.row_w + x) * rp.half;
+}
+// (cos, sin) of pair j: the frame's, the row's or the column's table row by the pair's group.
+__device__ __forceinline__ float2 rope_cs(const RopeDev& rp, int j, const float2* rt, const float2* rh,
+                                          const float2* rw) {
+  return __ldg((j < rp.pt ? rt : (j < rp.pth ? rh : rw)) + j);
+}
+__device__ __forceinline__ float2 turn_pair(float a, float b, float2 cs) {
+  return make_float2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
+}
+
+// Turns the feature pairs (2p, 2p + 1) of the first `rows` rows of a 128-row bf16 tile in place;
+// row i is token n0 + i. The tile is `natoms` swizzle-128B atoms of 64 features. The 128 threads of
+// the ReLU warps (index r) split it as in relu_tile_inplace: thread r owns the physical 16-byte
+// chunk r % 8 of the rows r / 8 + 16 m, which is the same logical chunk (4 pairs) in every such row.
+__device__ void rope_tile_inplace(uint8_t* tile, int natoms, int r, int n0, int rows, const RopeDev& rp) {
+  const int pc = r & 7;
+  const int rb = r >> 3;
+  const int lc = pc ^ (rb & 7);
+  for (int m = 0; m < 8; ++m) {
+    const int row = rb + 16 * m;
+    if (row >= rows) break;
+    const float2 *rt, *rh, *rw;
+    rope_rows(rp, n0 + row, rt, rh, rw);
+    for (int a = 0; a < natoms; ++a) {
+      const int j0 = 32 * a + 4 * lc;
+      if (j0 >= rp.half) continue;  // features beyond D (zero padding of the last atom)
+      uint4* p = reinterpret_cast<uint4*>(tile + a * kAtomBytes + row * 128 + (pc << 4));
+      uint4 x = *p;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+        const float2 t = turn_pair(ab.x, ab.y, rope_cs(rp, j0 + u, rt, rh, rw));
+        w[u] = pack_bf16x2(t.x, t.y);
+      }
+      *p = x;
+    }
   }
 }
 
@@ -225,8 +280,54 @@ __device__ void relu_role(uint8_t* smem, const Bars& b, long long tb, long long 
   }
 }
 
-__device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, uint32_t tmem,
-                         uint32_t* status) {
+// Rotary form only: per stage, the z products of a tile retired (the turn may overwrite the
+// features) and the tile turned (the S products may read it).
+struct RopeBars {
+  uint64_t* zd;   // [3] count 1 (tcgen05.commit)
+  uint64_t* rot;  // [3] count 4 (the ReLU warps)
+};
+constexpr int kRopeBars = 2 * kStages;
+__device__ __forceinline__ RopeBars rope_bars_at(uint64_t* p) { return RopeBars{p, p + kStages}; }
+__device__ __forceinline__ void init_rope_bars(const RopeBars& rb) {
+  for (int i = 0; i < kStages; ++i) {
+    mbar_init(&rb.zd[i], 1);
+    mbar_init(&rb.rot[i], 4);
+  }
+}
+
+// relu_role of the rotary form: ReLU of tile k, then the turn of tile k - 1 (whose z products the
+// MMA warp issued as soon as its ReLU was done, so they have had a tile's time to retire).
+__device__ void relu_rope_role(uint8_t* smem, const Bars& b, const RopeBars& rb, const Geom& geo, long long tb,
+                               long long te, bool two_atoms, int r, int lane, const RopeDev& rp, uint32_t* status) {
+  const int nchunks = (two_atoms ? kKBytes : kAtomBytes) / 16;
+  const auto turn = [&](int k, long long t) -> bool {
+    const int s = k % kStages;
+    const bool ok = mbar_wait(&rb.zd[s], (k / kStages) & 1, status, 0x0240u | s);
+    if (!warp_all(ok)) return false;
+    const TileCoord c = tile_coord(t, geo);
+    rope_tile_inplace(smem + s * kStageBytes, two_atoms ? 2 : 1, r, c.blk * geo.L + c.tok0, c.rows, rp);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&rb.rot[s]);
+    return true;
+  };
+  int k = 0;
+  for (long long t = tb; t < te; ++t, ++k) {
+    const int s = k % kStages;
+    bool ok = mbar_wait(&b.full[s], (k / kStages) & 1, status, 0x0200u | s);
+    if (!warp_all(ok)) return;
+    relu_tile_inplace(smem + s * kStageBytes, nchunks, r);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b.relu[s]);
+    if (k > 0 && !turn(k - 1, t - 1)) return;
+  }
+  if (k > 0) turn(k - 1, te - 1);
+}
+
+template <bool kRope>
+__device__ void mma_issue(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, uint32_t tmem,
+                          uint32_t* status, const RopeBars* rb) {
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, true, true);
   constexpr uint32_t kIdescZ = idesc_bf16_f32(128, 16, true, true);
   const uint64_t od = sdesc_sw128(smem_u32(smem + kOnesOff), kAtomBytes, 1024);  // same 16 rows of ones each step
@@ -245,14 +346,29 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long lon
     const uint32_t kb = smem_u32(smem + s * kStageBytes);
     const uint32_t vb = kb + kKBytes;
     const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
+    if constexpr (kRope) {
+      // z from the unturned ReLU(K), then S from the turned tile
 #pragma unroll
-    for (int kk = 0; kk < kTile / 16; ++kk) {
-      // 16 tokens per MMA: two groups of 8 token rows (128 B each) -> +2048 B per step
-      const uint64_t ad = sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024);
-      const uint64_t bd = sdesc_sw128(vb + kk * 2048, kAtomBytes, 1024);
-      const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-      mma_bf16(dacc, ad, bd, kIdescS, acc);         // S^T columns: ReLU(K)^T V
-      mma_bf16(dacc + 128, ad, od, kIdescZ, acc);   // z column: ReLU(K)^T 1
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16(dacc + 128, sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024), od, kIdescZ,
+                 (first && kk == 0) ? 0u : 1u);
+      mma_commit(&rb->zd[s]);
+      if (!mbar_wait(&rb->rot[s], ph, status, 0x0330u | s)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_bf16(dacc, sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024), sdesc_sw128(vb + kk * 2048, kAtomBytes, 1024),
+                 kIdescS, (first && kk == 0) ? 0u : 1u);
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        // 16 tokens per MMA: two groups of 8 token rows (128 B each) -> +2048 B per step
+        const uint64_t ad = sdesc_sw128(kb + kk * 2048, kAtomBytes, 1024);
+        const uint64_t bd = sdesc_sw128(vb + kk * 2048, kAtomBytes, 1024);
+        const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+        mma_bf16(dacc, ad, bd, kIdescS, acc);         // S^T columns: ReLU(K)^T V
+        mma_bf16(dacc + 128, ad, od, kIdescZ, acc);   // z column: ReLU(K)^T 1
+      }
     }
     mma_commit(&b.empty[s]);
     if (end) {
@@ -262,6 +378,10 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long lon
   }
   mma_commit(b.done);
   mbar_wait(b.done, 0, status, 0x03F0u);
+}
+__device__ __forceinline__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te,
+                                         uint32_t tmem, uint32_t* status) {
+  mma_issue<false>(smem, b, geo, tb, te, tmem, status, nullptr);
 }
 
 // Epilogue: warp w drains TMEM lanes 32w..32w+31 (key feature d) into the partial slot g + segment,
@@ -477,9 +597,26 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
   for (int i = (j > 2 ? j - 2 : 0); i < j; ++i) mbar_wait(&b.bfull[i & 1], (i >> 1) & 1, status, 0x1190u);
 }
 
-__device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, const Seq& sq, bool two_atoms, uint32_t tmem,
-                         uint32_t* status) {
+// Rotary form only: per stage, the denominator products of a Q tile retired, and the tile turned.
+struct RopeBars {
+  uint64_t* zd;   // [3] count 1 (tcgen05.commit)
+  uint64_t* rot;  // [3] count 4 (the ReLU warps)
+};
+constexpr int kRopeBars = 2 * kStages;
+__device__ __forceinline__ RopeBars rope_bars_at(uint64_t* p) { return RopeBars{p, p + kStages}; }
+__device__ __forceinline__ void init_rope_bars(const RopeBars& rb) {
+  for (int i = 0; i < kStages; ++i) {
+    mbar_init(&rb.zd[i], 1);
+    mbar_init(&rb.rot[i], 4);
+  }
+}
+
+template <bool kRope>
+__device__ void mma_issue(uint8_t* smem, const Bars& b, const Geom& geo, const Seq& sq, bool two_atoms, uint32_t tmem,
+                          uint32_t* status, const RopeBars* rb) {
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, kPTileRows, false, false);
+  constexpr uint32_t kIdescNum = idesc_bf16_f32(128, 128, false, false);
+  constexpr uint32_t kIdescDen = idesc_bf16_f32(128, 16, false, false);
   const int ksteps = two_atoms ? 8 : 4;
   int j = 0, prev = -1, bb = 0;
   for (int k = 0;; ++k) {
@@ -511,17 +648,36 @@ __device__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, const Se
     const uint32_t qb = smem_u32(smem + s * kQBytes);
     const uint32_t bbase = smem_u32(smem + kBOff + bb * kPTileBytes);
     const uint32_t dacc = tmem + static_cast<uint32_t>(a * 256);
-    for (int kk = 0; kk < ksteps; ++kk) {
-      // 16 features per MMA: +32 B inside the 128-B swizzle row, next atom after 4 steps
-      const uint64_t ad = sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024);
-      const uint64_t bd = sdesc_sw128(bbase + (kk >> 2) * kBAtomBytes + (kk & 3) * 32, 16, 1024);
-      mma_bf16(dacc, ad, bd, kIdescO, kk > 0 ? 1u : 0u);
+    if constexpr (kRope) {
+      // denominator from the unturned ReLU(Q) against the z row and its 15 zero rows (B rows
+      // 128..143, 16 KB into each atom), then the numerator from the turned tile against P^T
+      for (int kk = 0; kk < ksteps; ++kk)
+        mma_bf16(dacc + kZRow, sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(bbase + (kk >> 2) * kBAtomBytes + kZRow * 128 + (kk & 3) * 32, 16, 1024), kIdescDen,
+                 kk > 0 ? 1u : 0u);
+      mma_commit(&rb->zd[s]);
+      if (!mbar_wait(&rb->rot[s], ph, status, 0x1350u | s)) break;
+      tc_fence_after();
+      for (int kk = 0; kk < ksteps; ++kk)
+        mma_bf16(dacc, sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(bbase + (kk >> 2) * kBAtomBytes + (kk & 3) * 32, 16, 1024), kIdescNum, kk > 0 ? 1u : 0u);
+    } else {
+      for (int kk = 0; kk < ksteps; ++kk) {
+        // 16 features per MMA: +32 B inside the 128-B swizzle row, next atom after 4 steps
+        const uint64_t ad = sdesc_sw128(qb + (kk >> 2) * kAtomBytes + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(bbase + (kk >> 2) * kBAtomBytes + (kk & 3) * 32, 16, 1024);
+        mma_bf16(dacc, ad, bd, kIdescO, kk > 0 ? 1u : 0u);
+      }
     }
     mma_commit(&b.qempty[s]);
     mma_commit(&b.accf[a]);
   }
   mma_commit(b.done);
   mbar_wait(b.done, 0, status, 0x13F0u);
+}
+__device__ __forceinline__ void mma_role(uint8_t* smem, const Bars& b, const Geom& geo, const Seq& sq, bool two_atoms,
+                                         uint32_t tmem, uint32_t* status) {
+  mma_issue<false>(smem, b, geo, sq, two_atoms, tmem, status, nullptr);
 }
 
 // ReLU of the k-th Q tile (stage k % kStages) in place. Returns 1 when done, 0 at the end of the
@@ -641,6 +797,61 @@ __device__ void relu_epi_role(uint8_t* smem, const Staging& sg, const Bars& b, c
   }
   if (two_atoms && lane == 0) bulk_wait_all();
 }
+
+// Turn of the k-th Q tile once its denominator products retired. Returns 1, or -1 if the grid failed.
+__device__ __forceinline__ int turn_q(uint8_t* smem, const RopeBars& rb, const Geom& geo, const Seq& sq, long long k,
+                                      bool two_atoms, int r, int lane, const RopeDev& rp, uint32_t* status) {
+  const int s = static_cast<int>(k % kStages);
+  const bool ok = mbar_wait(&rb.zd[s], static_cast<uint32_t>((k / kStages) & 1), status, 0x1240u | s);
+  if (!warp_all(ok)) return -1;
+  const volatile int4* ent = sq.ring + (k % kRing);
+  const int blk = ent->z, tok0 = ent->w;
+  const int blen = blk == geo.nblk - 1 ? geo.Llast : geo.L;
+  rope_tile_inplace(smem + s * kQBytes, two_atoms ? 2 : 1, r, blk * geo.L + tok0, min(kTile, blen - tok0), rp);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&rb.rot[s]);
+  return 1;
+}
+
+// relu_epi_role of the rotary form: ReLU of tile k + kStages and the turn of tile k + kStages - 1
+// after the epilogue of tile k (one tile of lag between ReLU and turn, so that the denominator
+// products have retired). The turn of tile k + 2 waits for the MMA warp's denominator products,
+// which wait for the accumulator that the epilogue of tile k released, so the order cannot
+// deadlock; at the end of the sequence every ReLU'd tile is turned.
+__device__ void relu_rot_epi_role(uint8_t* smem, const Staging& sg, const Bars& b, const RopeBars& rb, const Maps4& m,
+                                  const Geom& geo, const Seq& sq, bool two_atoms, uint32_t tmem, int warp, int lane,
+                                  float eps, const RopeDev& rp, uint32_t* status) {
+  const int r = static_cast<int>(threadIdx.x) - 128;
+  long long kr = 0, kq = 0;  // tiles ReLU'd, tiles turned
+  int rs = 1;                // 1 more tiles, 0 sequence ended, -1 failed
+  const auto relu_next = [&]() {
+    if (rs > 0) {
+      rs = relu_q(smem, b, sq, kr, two_atoms, r, lane, status);
+      if (rs > 0) ++kr;
+    }
+  };
+  const auto turn_upto = [&](long long upto) -> bool {
+    for (; kq < kr && kq < upto; ++kq)
+      if (turn_q(smem, rb, geo, sq, kq, two_atoms, r, lane, rp, status) < 0) return false;
+    return true;
+  };
+  for (int i = 0; i < kStages; ++i) {
+    relu_next();
+    if (rs < 0 || !turn_upto(rs == 0 ? kr : i)) return;
+  }
+  for (long long k = 0;; ++k) {
+    if (two_atoms) {
+      const int es = epilogue_tile(sg, b, m, geo, sq, k, tmem, warp & 3, 1, lane, eps, status);
+      if (es <= 0) break;
+    } else if (rs == 0 && kq == kr) {
+      break;
+    }
+    relu_next();
+    if (rs < 0 || !turn_upto(rs == 0 ? kr : k + kStages)) break;
+  }
+  if (two_atoms && lane == 0) bulk_wait_all();
+}
 }  // namespace ot
 
 // ---- common prologue / epilogue of the persistent kernels ----
@@ -678,16 +889,21 @@ constexpr int kOutSmem = ot::kRegionBytes + 1024 + 512 + 1024;
 static_assert((ot::kNumBars + 2) * 8 + ot::kRingBytes <= 512, "output kernel barrier area");
 static_assert((st::kNumBars + ot::kNumBars + 2) * 8 + ot::kRingBytes <= 512, "single-launch barrier area");
 
+static_assert((st::kNumBars + 1 + st::kRopeBars) * 8 <= 256, "state kernel barrier area");
+static_assert((ot::kNumBars + 2) * 8 + ot::kRingBytes + ot::kRopeBars * 8 <= 512, "output kernel barrier area (rotary)");
+
+template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     state_bf16_kernel(const __grid_constant__ CUtensorMap k_main, const __grid_constant__ CUtensorMap k_last,
                       const __grid_constant__ CUtensorMap v_main, const __grid_constant__ CUtensorMap v_last,
                       const Geom geo, float* __restrict__ partials, int2* __restrict__ segcta,
-                      uint32_t* status) {
+                      uint32_t* status, const RopeDev rp) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + st::kRegionBytes);
   const st::Bars b = st::bars_at(barmem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + st::kNumBars);
+  const st::RopeBars rb = st::rope_bars_at(barmem + st::kNumBars + 1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -697,6 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Maps4 m{&k_main, &k_last, &v_main, &v_last};
   if (threadIdx.x == 0) {
     st::init_bars(b);
+    if (kRope) st::init_rope_bars(rb);
     fence_mbar_init();
   }
   st::init_smem(smem, two_atoms, kThreads);
@@ -706,25 +923,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpProducer) {
     if (lane == 0) st::produce(smem, b, m, geo, tb, te, two_atoms, true, status);
   } else if (warp >= 4 && warp < 8) {
-    st::relu_role(smem, b, tb, te, two_atoms, threadIdx.x - 128, lane, status);
+    if constexpr (kRope)
+      st::relu_rope_role(smem, b, rb, geo, tb, te, two_atoms, threadIdx.x - 128, lane, rp, status);
+    else
+      st::relu_role(smem, b, tb, te, two_atoms, threadIdx.x - 128, lane, status);
   } else if (warp == kWarpMma) {
-    if (lane == 0) st::mma_role(smem, b, geo, tb, te, tmem, status);
+    if (lane == 0) st::mma_issue<kRope>(smem, b, geo, tb, te, tmem, status, &rb);
   } else {
     st::epilogue_role(b, geo, tb, te, tmem, g, warp, lane, partials, segcta, nullptr, nullptr, 0, status);
   }
   persistent_teardown(tmem, warp);
 }
 
+template <bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     out_bf16_kernel(const __grid_constant__ CUtensorMap q_main, const __grid_constant__ CUtensorMap q_last,
                     const __grid_constant__ CUtensorMap o_main, const __grid_constant__ CUtensorMap o_last,
-                    const Geom geo, const uint8_t* __restrict__ ptiles, const float eps, uint32_t* status) {
+                    const Geom geo, const uint8_t* __restrict__ ptiles, const float eps, uint32_t* status,
+                    const RopeDev rp) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* barmem = reinterpret_cast<uint64_t*>(smem + ot::kRegionBytes);
   const ot::Bars b = ot::bars_at(barmem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barmem + ot::kNumBars);
   volatile int4* ring = reinterpret_cast<volatile int4*>(barmem + ot::kNumBars + 2);  // 16-byte aligned
+  const ot::RopeBars rb = ot::rope_bars_at(barmem + ot::kNumBars + 2 + ot::kRingBytes / 8);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -735,6 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Maps4 m{&q_main, &q_last, &o_main, &o_last};
   if (threadIdx.x == 0) {
     ot::init_bars(b, two_atoms);
+    if (kRope) ot::init_rope_bars(rb);
     fence_mbar_init();
   }
   if (warp == kWarpProducer && lane == 0) prefetch_maps(m);
@@ -747,10 +971,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ot::produce(smem, b, m, geo, sq, pre, two_atoms, ptiles, nullptr, 0, status);
     }
   } else if (warp >= 4 && warp < 8) {
-    ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, 0, two_atoms, tmem, warp, lane, eps,
-                      status);
+    if constexpr (kRope)
+      ot::relu_rot_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, rb, m, geo, sq, two_atoms, tmem, warp, lane,
+                            eps, rp, status);
+    else
+      ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, 0, two_atoms, tmem, warp, lane, eps,
+                        status);
   } else if (warp == kWarpMma) {
-    if (lane == 0) ot::mma_role(smem, b, geo, sq, two_atoms, tmem, status);
+    if (lane == 0) ot::mma_issue<kRope>(smem, b, geo, sq, two_atoms, tmem, status, &rb);
   } else {
     ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, tmem, warp, lane, eps, status);
   }
@@ -1792,13 +2020,33 @@ __device__ __forceinline__ float relu_f32(float x) { return (x != x) ? x : fmaxf
 constexpr int kF32Threads = 256;
 constexpr int kStateF32Smem = 2 * kTile * kDPad * 4;                   // K, V tiles
 constexpr int kOutF32Smem = kDPad * kPartRows * 4 + kTile * kDPad * 4;  // prefix (transposed), Q tile
+constexpr int kF32TurnedBytes = kTile * kDPad * 4;                      // rotary form: the turned tile
+
+// Rotary form: Xt = the feature pairs of the first `rows` rows of X turned (rows beyond: zero).
+__device__ void turn_tile_f32(const float* X, float* Xt, int rows, int n0, int D, const RopeDev& rp) {
+  const int half = D / 2;
+  for (int i = threadIdx.x; i < kTile * half; i += kF32Threads) {
+    const int rr = i / half, jj = i - rr * half;
+    float2 t = make_float2(0.f, 0.f);
+    if (rr < rows) {
+      const float2 *rt, *rh, *rw;
+      rope_rows(rp, n0 + rr, rt, rh, rw);
+      t = turn_pair(X[rr * kDPad + 2 * jj], X[rr * kDPad + 2 * jj + 1], rope_cs(rp, jj, rt, rh, rw));
+    }
+    Xt[rr * kDPad + 2 * jj] = t.x;
+    Xt[rr * kDPad + 2 * jj + 1] = t.y;
+  }
+}
 
 __global__ void __launch_bounds__(kF32Threads, 1)
     state_f32_kernel(const float* __restrict__ k, const float* __restrict__ v, const Geom geo,
-                     float* __restrict__ partials, int2* __restrict__ segcta) {
+                     float* __restrict__ partials, int2* __restrict__ segcta, const RopeDev rp) {
   extern __shared__ float fsm[];
   float* Ks = fsm;
   float* Vs = fsm + kTile * kDPad;
+  float* Kt = fsm + 2 * kTile * kDPad;  // rotary form only
+  const bool rope = rp.tab != nullptr;
+  const float* KS = rope ? Kt : Ks;     // the S products read the turned features, z the unturned
   const int D = geo.D;
   const int d = threadIdx.x & 127;
   const int eh = threadIdx.x >> 7;
@@ -1820,10 +2068,14 @@ __global__ void __launch_bounds__(kF32Threads, 1)
       Vs[rr * kDPad + cc] = in ? v[row0 * D + i] : 0.f;
     }
     __syncthreads();
+    if (rope) {
+      turn_tile_f32(Ks, Kt, c.rows, c.blk * geo.L + c.tok0, D, rp);
+      __syncthreads();
+    }
     if (d < D) {
       for (int jr = 0; jr < c.rows; ++jr) {
-        const float fk = Ks[jr * kDPad + d];
-        if (eh == 0) zacc += fk;
+        if (eh == 0) zacc += Ks[jr * kDPad + d];
+        const float fk = KS[jr * kDPad + d];
 #pragma unroll
         for (int m = 0; m < 64; ++m) {
           const int e = eh + 2 * m;
@@ -1851,10 +2103,13 @@ __global__ void __launch_bounds__(kF32Threads, 1)
 
 __global__ void __launch_bounds__(kF32Threads, 1)
     out_f32_kernel(const float* __restrict__ q, float* __restrict__ o, const Geom geo,
-                   const float* __restrict__ p32, const float eps) {
+                   const float* __restrict__ p32, const float eps, const RopeDev rp) {
   extern __shared__ float fsm[];
   float* Ps = fsm;                      // [d][e'] with e' = 0..128 (z at 128)
   float* Qs = fsm + kDPad * kPartRows;  // [row][d]
+  float* Qt = Qs + kTile * kDPad;       // rotary form only: the turned tile
+  const bool rope = rp.tab != nullptr;
+  const float* QN = rope ? Qt : Qs;     // the numerator reads the turned features, the denominator the unturned
   const int D = geo.D;
   const int g = blockIdx.x;
   const long long tb = tile_begin(g, geo);
@@ -1879,20 +2134,51 @@ __global__ void __launch_bounds__(kF32Threads, 1)
       Qs[rr * kDPad + cc] = rr < c.rows ? relu_f32(q[row0 * D + i]) : 0.f;
     }
     __syncthreads();
+    if (rope) {
+      turn_tile_f32(Qs, Qt, c.rows, c.blk * geo.L + c.tok0, D, rp);
+      __syncthreads();
+    }
     if (e < D) {
       for (int m = 0; m < 64; ++m) {
         const int rr = rh + 2 * m;
         if (rr >= c.rows) break;
         float num = 0.f, den = 0.f;
         for (int dd = 0; dd < D; ++dd) {
-          const float fq = Qs[rr * kDPad + dd];
-          num = fmaf(fq, Ps[dd * kPartRows + e], num);
-          den = fmaf(fq, Ps[dd * kPartRows + kZRow], den);
+          num = fmaf(QN[rr * kDPad + dd], Ps[dd * kPartRows + e], num);
+          den = fmaf(Qs[rr * kDPad + dd], Ps[dd * kPartRows + kZRow], den);
         }
         o[(row0 + rr) * D + e] = num / (den + eps);
       }
     }
   }
+}
+
+// (cos, sin) table of the rotary form: one thread per (row, pair). Row < frames: frame position
+// row; then `height` grid rows, then `width` grid columns. Pair j of a group of P pairs starting
+// at pair `off` turns by pos * base^(-(j - off) / P) (fp64 angle, rounded to fp32 once); pairs of
+// the other groups hold (1, 0).
+__global__ void rope_table_kernel(float2* tab, int frames, int height, int width, int half, int pt, int ph, int pw,
+                                  double base) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<long long>(frames + height + width) * half) return;
+  const int row = static_cast<int>(i / half);
+  const int j = static_cast<int>(i - static_cast<long long>(row) * half);
+  int pos, off, P;
+  if (row < frames) {
+    pos = row, off = 0, P = pt;
+  } else if (row < frames + height) {
+    pos = row - frames, off = pt, P = ph;
+  } else {
+    pos = row - frames - height, off = pt + ph, P = pw;
+  }
+  float2 cs = make_float2(1.f, 0.f);
+  if (j >= off && j < off + P) {
+    const double ang = static_cast<double>(pos) * pow(base, -static_cast<double>(j - off) / P);
+    double sn, cn;
+    sincos(ang, &sn, &cn);
+    cs = make_float2(static_cast<float>(cn), static_cast<float>(sn));
+  }
+  tab[i] = cs;
 }
 
 }  // namespace
@@ -1926,29 +2212,49 @@ size_t out_f32_smem_bytes() { return kOutF32Smem; }
 
 cudaError_t set_kernel_attributes() {
   cudaError_t e;
-  e = cudaFuncSetAttribute(state_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+  e = cudaFuncSetAttribute(state_bf16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(state_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(out_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fu::kSmem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(cluster_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cl::kSmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(out_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+  e = cudaFuncSetAttribute(out_bf16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(state_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateF32Smem);
+  e = cudaFuncSetAttribute(state_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kStateF32Smem + kF32TurnedBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(out_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutF32Smem);
+  return cudaFuncSetAttribute(out_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kOutF32Smem + kF32TurnedBytes);
 }
 
 cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,
-                              uint32_t* status, cudaStream_t s) {
-  return launch_pdl(state_bf16_kernel, dim3(g.G), dim3(kThreads), kStateSmem, s, k.main, k.last, v.main, v.last,
-                    g, partials, segcta, status);
+                              uint32_t* status, cudaStream_t s, const RopeDev* rope) {
+  if (rope != nullptr)
+    return launch_pdl(state_bf16_kernel<true>, dim3(g.G), dim3(kThreads), kStateSmem, s, k.main, k.last, v.main,
+                      v.last, g, partials, segcta, status, *rope);
+  return launch_pdl(state_bf16_kernel<false>, dim3(g.G), dim3(kThreads), kStateSmem, s, k.main, k.last, v.main,
+                    v.last, g, partials, segcta, status, RopeDev{});
 }
 
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles, float eps,
-                            uint32_t* status, cudaStream_t s) {
-  return launch_pdl(out_bf16_kernel, dim3(g.G), dim3(kThreads), kOutSmem, s, q.main, q.last, o.main, o.last,
-                    g, static_cast<const uint8_t*>(ptiles), eps, status);
+                            uint32_t* status, cudaStream_t s, const RopeDev* rope) {
+  if (rope != nullptr)
+    return launch_pdl(out_bf16_kernel<true>, dim3(g.G), dim3(kThreads), kOutSmem, s, q.main, q.last, o.main, o.last,
+                      g, static_cast<const uint8_t*>(ptiles), eps, status, *rope);
+  return launch_pdl(out_bf16_kernel<false>, dim3(g.G), dim3(kThreads), kOutSmem, s, q.main, q.last, o.main, o.last,
+                    g, static_cast<const uint8_t*>(ptiles), eps, status, RopeDev{});
+}
+
+cudaError_t launch_rope_table(float2* tab, int frames, int height, int width, int half, int pt, int ph, int pw,
+                              double base, cudaStream_t s) {
+  const long long n = static_cast<long long>(frames + height + width) * half;
+  rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(tab, frames, height, width, half, pt, ph,
+                                                                           pw, base);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_fused_bf16(const BlockMaps& k, const BlockMaps& v, const BlockMaps& q, const BlockMaps& o,
@@ -2068,14 +2374,16 @@ cudaError_t launch_scan(const float* partials, const int2* segcta, const Geom& g
 }
 
 cudaError_t launch_state_f32(const float* k, const float* v, const Geom& g, float* partials, int2* segcta,
-                             uint32_t*, cudaStream_t s) {
-  state_f32_kernel<<<g.G, kF32Threads, kStateF32Smem, s>>>(k, v, g, partials, segcta);
+                             uint32_t*, cudaStream_t s, const RopeDev* rope) {
+  const int smem = kStateF32Smem + (rope != nullptr ? kF32TurnedBytes : 0);
+  state_f32_kernel<<<g.G, kF32Threads, smem, s>>>(k, v, g, partials, segcta, rope != nullptr ? *rope : RopeDev{});
   return cudaGetLastError();
 }
 
 cudaError_t launch_out_f32(const float* q, float* o, const Geom& g, const float* p32, float eps, uint32_t*,
-                           cudaStream_t s) {
-  out_f32_kernel<<<g.G, kF32Threads, kOutF32Smem, s>>>(q, o, g, p32, eps);
+                           cudaStream_t s, const RopeDev* rope) {
+  const int smem = kOutF32Smem + (rope != nullptr ? kF32TurnedBytes : 0);
+  out_f32_kernel<<<g.G, kF32Threads, smem, s>>>(q, o, g, p32, eps, rope != nullptr ? *rope : RopeDev{});
   return cudaGetLastError();
 }
 

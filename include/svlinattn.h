@@ -165,6 +165,54 @@ sv_status sv_cache_step_noalloc(const void* q, const void* k, const void* v, voi
  * the word in *code if given). Allocates nothing. */
 sv_status sv_cache_step_noalloc_status(sv_stream_t stream, uint32_t* code);
 
+/* 3D rotary position embedding inside the linear attention (talk, passage on adapting the Linear
+ * DiT to video: 3D RoPE for the linear attention; model-family page, architecture paragraph:
+ * rotary position embeddings). The pages print no formula; this library reads it as follows.
+ *  - The rotation acts on the feature-mapped q and k. It is applied to the numerator only; the
+ *    normaliser keeps the unturned features, so that it stays positive:
+ *        o_i = R_i phi(q_i) . P / (phi(q_i) . zP + eps),
+ *        P = S_in + sum_j (R_j phi(k_j)) v_j^T,   zP = z_in + sum_j phi(k_j)   (visible j).
+ *  - R_n turns the feature pairs (2p, 2p+1) by the angle pos * base^(-p'/P): the D/2 pairs are
+ *    split into groups of pairs_t, pairs_h, pairs_w pairs (in that order) that take the token's
+ *    frame, grid row and grid column as pos; p' is the pair's index in its group of P pairs.
+ *  - Tokens are flattened frame-major on a grid of height x width tokens per frame: token n of a
+ *    (batch, head) sequence sits at frame frame0 + n / (height*width), row (n / width) % height,
+ *    column n % width.
+ * The (cos, sin) table is built once per grid and feature split. */
+typedef struct {
+  const float* table; /* DEVICE table written by sv_rope3d_table with the fields below */
+  int frames;         /* frame positions the table covers (0 .. frames-1) */
+  int height, width;  /* tokens per frame: height rows x width columns */
+  int D;              /* feature dimension of the table (even) */
+  int pairs_t, pairs_h, pairs_w; /* pairs per group; 2 * (pairs_t + pairs_h + pairs_w) == D */
+  int frame0;         /* frame of token 0 of q and k in the call; the call's last token must sit
+                         inside the table: frame0 + (N-1) / (height*width) < frames */
+} sv_rope3d;
+
+/* Bytes of the table for `frames` frame positions, a height x width grid and feature dimension D:
+ * (frames + height + width) * (D/2) * 8. 0 for arguments out of range (see sv_last_error). */
+size_t sv_rope3d_table_bytes(int frames, int height, int width, int D);
+
+/* Writes the (cos, sin) table into `table` (DEVICE, 16-byte aligned, table_bytes >=
+ * sv_rope3d_table_bytes(...)): rows 0..frames-1 are frame positions, then `height` rows, then
+ * `width` columns; each row holds D/2 fp32 (cos, sin) pairs, the angle of pair p' of the row's
+ * group being pos * base^(-p'/P) computed in fp64 and rounded once; pairs of the other groups hold
+ * (1, 0). base > 1 (10000 in RoFormer). One kernel on `stream`. */
+sv_status sv_rope3d_table(float* table, size_t table_bytes, int frames, int height, int width, int D, int pairs_t,
+                          int pairs_h, int pairs_w, float base, sv_stream_t stream);
+
+/* sv_block_causal_attn with the 3D rotary embedding above (rope: HOST pointer to the descriptor,
+ * read during the call). Arguments, outputs and the workspace (sv_workspace_bytes with
+ * SV_OP_BLOCK_CAUSAL_ATTN) are those of sv_block_causal_attn. S_in / S_out hold the turned-key
+ * state, z_in / z_out the unturned key sum, so one streaming step of the cache is this call with
+ * block_len = N, S_in = S_out = S, z_in = z_out = z, and frame0 = the block's first frame;
+ * block_len >= N is the bidirectional form. D must be even. The work always runs as the
+ * three-kernel path (state, scan, output), also for one block per head. */
+sv_status sv_block_causal_attn_rope(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int D,
+                                    int block_len, sv_dtype dt, float eps, const float* S_in, const float* z_in,
+                                    float* S_out, float* z_out, const sv_rope3d* rope, void* ws, size_t ws_bytes,
+                                    sv_stream_t stream);
+
 /* Block-causal temporal convolution of the causal Mix-FFN (talk, causal FFN with temporal conv
  * passage: a zero token is padded between two blocks so that block 1 cannot see block 2, and block
  * 2 takes block 1's last token as its first token so that it sees block 1; the padding and the

@@ -74,6 +74,38 @@ def test_validation_rejects_before_any_launch(lib):
     assert lib.sv_workspace_init(None, 0, None) == 1
 
 
+def test_rope_arguments_are_checked_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    from block_causal_linear_relu_b200._native import SvRope3d
+
+    assert lib.sv_rope3d_table_bytes(60, 23, 40, 128) == (60 + 23 + 40) * 64 * 8
+    assert lib.sv_rope3d_table_bytes(60, 23, 40, 127) == 0 and b"even" in lib.sv_last_error()
+    assert lib.sv_rope3d_table_bytes(0, 23, 40, 128) == 0
+    fake = vp(256 * 1024)
+    tab = lib.sv_rope3d_table
+    n = (60 + 23 + 40) * 64 * 8
+    assert tab(fake, n, 60, 23, 40, 128, 22, 21, 20, 10000.0, None) == 1  # pairs sum to 63, not 64
+    assert b"pairs" in lib.sv_last_error()
+    assert tab(fake, n - 8, 60, 23, 40, 128, 22, 21, 21, 10000.0, None) == 1  # table too small
+    assert tab(fake, n, 60, 23, 40, 128, 22, 21, 21, 1.0, None) == 1  # base must exceed 1
+    assert tab(vp(256 * 1024 + 8), n, 60, 23, 40, 128, 22, 21, 21, 10000.0, None) == 1  # misaligned
+    f = lib.sv_block_causal_attn_rope
+
+    def call(desc, N=2760 * 3, D=128):
+        return f(fake, fake, fake, fake, 1, 20, N, D, 2760, 0, 1e-6, None, None, None, None,
+                 None if desc is None else ctypes.byref(desc), fake, 1 << 30, None)
+
+    good = dict(table=256 * 1024, frames=9, height=23, width=40, D=128, pairs_t=22, pairs_h=21, pairs_w=21, frame0=0)
+    assert call(None) == 1 and b"NULL" in lib.sv_last_error()
+    assert call(SvRope3d(**{**good, "frame0": 1})) == 1  # tokens reach frame 9 of a 9-frame table
+    assert b"frame0" in lib.sv_last_error()
+    assert call(SvRope3d(**{**good, "D": 112})) == 1  # table built for another D
+    assert call(SvRope3d(**{**good, "pairs_w": 20})) == 1
+    assert call(SvRope3d(**{**good, "table": 256 * 1024 + 8})) == 1
+    assert call(SvRope3d(**{**good, "height": 0})) == 1
+    assert call(SvRope3d(**good), D=100) == 2  # bf16 D must be a multiple of 8 (checked first)
+
+
 def test_binding_rejects_bad_tensors_before_the_library():
     # the binding's single pass of checks: host tensors, wrong rank, mismatched shape or dtype and
     # non-contiguous tensors raise before any library or CUDA call
