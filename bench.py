@@ -400,7 +400,14 @@ EXTRA_WORKLOADS = {
                      "denoise", 48),
     "sv2_stack": ("SANA-Video 2.0-shaped stack: 24 bidirectional layers of B=2 H=20 N=10120 D=128, fresh inputs "
                   "per layer, back to back on one stream", 2, 20, 10120, 128, 10120, "fwd", 24),
+    "720p_prefill_rope": ("720p block-causal prefill with the 3D rotary embedding on the numerator: B=1 H=20 "
+                          "N=55200 (20 blocks of 3 frames of 23x40 tokens) D=128, pairs (22, 21, 21), "
+                          "sv_block_causal_attn_rope", 1, 20, 55200, 128, 2760, "rope", 4),
+    "720p_stream_rope": ("cache streaming with the 3D rotary embedding: 60 blocks of B=1 H=20 N=2760 (3 frames of "
+                         "23x40) D=128 through the fp32 cache, frame0 = 3 x block, one sv_block_causal_attn_rope "
+                         "per block", 1, 20, 2760, 128, 2760, "rope_stream", 60),
 }
+ROPE_GRID = (23, 40)  # tokens per 720p latent frame: rows x columns
 
 
 def _cpu_model():
@@ -435,8 +442,13 @@ def time_workload(name, passes: int, dev_index: int = 0):
     outs = [torch.empty_like(x[0]) for x in sets]
     S = torch.zeros(b, h, d, d, device=dev)
     z = torch.zeros(b, h, d, device=dev)
-    op = sv.SV_OP_LINATTN_FWD if kind == "fwd" else sv.SV_OP_CACHE_STEP
-    ws = sv.make_workspace(op, sets[0][0])
+    if kind.startswith("rope"):
+        ws = sv.make_workspace(sv.SV_OP_BLOCK_CAUSAL_ATTN, sets[0][0], blen)
+        fpb = n // (ROPE_GRID[0] * ROPE_GRID[1])  # frames per call
+        tab = sv.sv_rope3d_table(fpb * (reps if kind == "rope_stream" else 1), ROPE_GRID[0], ROPE_GRID[1], d,
+                                 sv.rope_pairs(d), device=dev)
+    else:
+        ws = sv.make_workspace(sv.SV_OP_LINATTN_FWD if kind == "fwd" else sv.SV_OP_CACHE_STEP, sets[0][0])
     stream = torch.cuda.current_stream()
     steps_per_block = 4 if kind == "denoise" else 1
 
@@ -444,6 +456,11 @@ def time_workload(name, passes: int, dev_index: int = 0):
         q, k, v = sets[i]
         if kind == "fwd":
             sv.sv_linattn_fwd(q, k, v, o=outs[i], ws=ws, stream=st)
+        elif kind == "rope":
+            sv.sv_block_causal_attn_rope(q, k, v, blen, tab, o=outs[i], ws=ws, stream=st)
+        elif kind == "rope_stream":  # block i sits at frames 3i .. 3i + 2 of the video
+            sv.sv_block_causal_attn_rope(q, k, v, n, tab, frame0=i * fpb, o=outs[i], S_in=S, z_in=z, S_out=S,
+                                         z_out=z, ws=ws, stream=st)
         else:  # a block's last step commits its state to the cache
             sv.sv_cache_step(q, k, v, S, z, commit=(i % steps_per_block == steps_per_block - 1), o=outs[i], ws=ws,
                              stream=st)
@@ -486,7 +503,7 @@ def time_workload(name, passes: int, dev_index: int = 0):
     tokheads = b * h * n
     call_bytes = tokheads * 4 * d * 2
     t_roof_ms = call_bytes / (hbm_gbs * 1e9) * 1e3
-    gl = 3 if blen < n else 1
+    gl = 3 if blen < n or kind.startswith("rope") else 1
     return {
         "workload": desc, "B": b, "H": h, "N": n, "D": d, "block_len": blen, "calls_per_pass": reps,
         "passes": passes, "kernels_per_call": gl, "gpu_launches": gl * reps * passes * 2,
@@ -503,7 +520,8 @@ def time_workload(name, passes: int, dev_index: int = 0):
 
 # passes of each other configuration timed inside the default bench run (each pass: every call of
 # the workload once, with distinct inputs)
-EXTRA_PASSES = {"480p_bidir": 200, "720p_stream": 5, "sv2_stack": 8, "720p_denoise": 4}
+EXTRA_PASSES = {"480p_bidir": 200, "720p_stream": 5, "sv2_stack": 8, "720p_denoise": 4, "720p_prefill_rope": 5,
+                "720p_stream_rope": 3}
 
 
 def time_conv(passes: int, dev_index: int = 0):

@@ -20,6 +20,7 @@ from ._native import (  # noqa: F401
     lib_path,
     load,
     make_workspace,
+    rope_pairs,
     sv_block_causal_attn,
     sv_block_causal_attn_rope,
     sv_block_state_update,

@@ -381,6 +381,13 @@ def sv_out_projection(o, w_o, y=None, ws: Workspace | None = None, stream=None):
     return y
 
 
+def rope_pairs(D: int):
+    """A split of the D/2 rotation pairs over (frame, row, column): row and column get D // 6 pairs
+    each, the frame axis the rest (22, 21, 21 for D = 128)."""
+    ph = D // 6
+    return (D // 2 - 2 * ph, ph, ph)
+
+
 def sv_rope3d_table_bytes(frames: int, height: int, width: int, D: int) -> int:
     n = load().sv_rope3d_table_bytes(frames, height, width, D)
     if n == 0:

@@ -393,6 +393,11 @@ sv_status rope_for(sv::RopeDev& rd, const sv_rope3d* r, int N, int D) {
   rd.row_w = r->frames + r->height;
   rd.pt = r->pairs_t;
   rd.pth = r->pairs_t + r->pairs_h;
+  rd.nf = static_cast<int>((static_cast<long long>(N) - 1) / hw) + 1;
+  rd.h = r->height;
+  const long long entries = static_cast<long long>(rd.nf) * r->pairs_t + static_cast<long long>(r->height) * r->pairs_h +
+                            static_cast<long long>(r->width) * r->pairs_w;
+  rd.compact = entries <= sv::kRopeSmemEntries ? static_cast<int>(entries) : 0;
   return SV_OK;
 }
 

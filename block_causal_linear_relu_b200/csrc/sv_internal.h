@@ -32,10 +32,17 @@ struct BlockMaps {
 // positions, [row_h, row_w) grid rows, [row_w, ...) grid columns; `half` = D / 2 pairs per row.
 // Token n of a (batch, head) sequence sits at frame f0 + n / hw, row (n % hw) / w, column n % w.
 // Pairs [0, pt) turn with the frame, [pt, pth) with the row, [pth, half) with the column.
+// The kernels of the bf16 path first copy the part of the table the call reads into shared
+// memory, in a compact form: for each of the nf frames the call's tokens touch (f0 .. f0 + nf - 1)
+// the frame group's pt pairs, then for each of the h grid rows the row group's pairs, then for
+// each of the w columns the column group's pairs. `compact` is that entry count, or 0 when it
+// exceeds kRopeSmemEntries (the kernels then read the table in global memory).
 struct RopeDev {
   const float2* tab;
   int half, hw, w, f0, row_h, row_w, pt, pth;
+  int nf, h, compact;
 };
+constexpr int kRopeSmemEntries = 3072;  // 24 KB of (cos, sin) pairs
 
 // bf16 path (rope: nullptr, or the rotation of the numerator's features)
 cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,

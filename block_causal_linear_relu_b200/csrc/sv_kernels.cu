@@ -65,7 +65,52 @@ __device__ __forceinline__ void relu_tile_inplace(uint8_t* tile, int nchunks, in
 }
 
 // ---- 3D rotary embedding of the feature-mapped features (numerator of the rotated form) ----
-// Table rows of token n's frame, grid row and grid column.
+// Copies the compact table (RopeDev) into shared memory at `ct`, by `nthreads` threads (index i0).
+// The table may come from the previous kernel in the stream: the caller has passed griddepcontrol.wait.
+__device__ void stage_rope_table(float2* ct, const RopeDev& rp, int i0, int nthreads) {
+  const int ph = rp.pth - rp.pt, pw = rp.half - rp.pth;
+  const int e_t = rp.nf * rp.pt, e_h = e_t + rp.h * ph;
+  for (int i = i0; i < rp.compact; i += nthreads) {
+    int row, j;
+    if (i < e_t) {
+      row = rp.f0 + i / rp.pt, j = i % rp.pt;
+    } else if (i < e_h) {
+      row = rp.row_h + (i - e_t) / ph, j = rp.pt + (i - e_t) % ph;
+    } else {
+      row = rp.row_w + (i - e_h) / pw, j = rp.pth + (i - e_h) % pw;
+    }
+    ct[i] = __ldg(rp.tab + static_cast<size_t>(row) * rp.half + j);
+  }
+}
+__device__ __forceinline__ float2 ld_shared_f2(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void st_shared_u4(uint32_t a, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+// Shared-memory byte addresses such that pair j of token n's frame / row / column group sits at
+// base + 8 j in the compact table at `ct` (each group's entries start at its first pair).
+__device__ __forceinline__ void rope_rows_smem(const RopeDev& rp, uint32_t ct, int n, uint32_t& bt, uint32_t& bh,
+                                               uint32_t& bw) {
+  const int f = n / rp.hw;
+  const int rem = n - f * rp.hw;
+  const int y = rem / rp.w;
+  const int x = rem - y * rp.w;
+  const int ph = rp.pth - rp.pt, pw = rp.half - rp.pth;
+  const int e_t = rp.nf * rp.pt;
+  bt = ct + 8u * static_cast<uint32_t>(f * rp.pt);
+  bh = ct + 8u * static_cast<uint32_t>(e_t + y * ph - rp.pt);
+  bw = ct + 8u * static_cast<uint32_t>(e_t + rp.h * ph + x * pw - rp.pth);
+}
+// Table rows of token n's frame, grid row and grid column (the table in global memory).
 __device__ __forceinline__ void rope_rows(const RopeDev& rp, int n, const float2*& rt, const float2*& rh,
                                           const float2*& rw) {
   const int f = n / rp.hw;
@@ -85,33 +130,80 @@ __device__ __forceinline__ float2 turn_pair(float a, float b, float2 cs) {
   return make_float2(fmaf(a, cs.x, -b * cs.y), fmaf(a, cs.y, b * cs.x));
 }
 
-// Turns the feature pairs (2p, 2p + 1) of the first `rows` rows of a 128-row bf16 tile in place;
-// row i is token n0 + i. The tile is `natoms` swizzle-128B atoms of 64 features. The 128 threads of
-// the ReLU warps (index r) split it as in relu_tile_inplace: thread r owns the physical 16-byte
-// chunk r % 8 of the rows r / 8 + 16 m, which is the same logical chunk (4 pairs) in every such row.
-__device__ void rope_tile_inplace(uint8_t* tile, int natoms, int r, int n0, int rows, const RopeDev& rp) {
-  const int pc = r & 7;
-  const int rb = r >> 3;
-  const int lc = pc ^ (rb & 7);
-  for (int m = 0; m < 8; ++m) {
-    const int row = rb + 16 * m;
-    if (row >= rows) break;
-    const float2 *rt, *rh, *rw;
-    rope_rows(rp, n0 + row, rt, rh, rw);
-    for (int a = 0; a < natoms; ++a) {
-      const int j0 = 32 * a + 4 * lc;
-      if (j0 >= rp.half) continue;  // features beyond D (zero padding of the last atom)
-      uint4* p = reinterpret_cast<uint4*>(tile + a * kAtomBytes + row * 128 + (pc << 4));
-      uint4 x = *p;
-      uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+// M consecutive 16-byte chunks c0 .. c0 + M - 1 (one atom) of one tile row at `arow`: every load
+// of the group is issued before the first use; straight-line code for the compiler to schedule.
+template <bool kSmem, int M>
+__device__ __forceinline__ void turn_group(uint32_t arow, int c0, int r7, int pt, int pth, uint32_t bt, uint32_t bh,
+                                           uint32_t bw, const float2* rt, const float2* rh, const float2* rw) {
+  uint4 x[M];
+  float2 cs[M][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
-        const float2 t = turn_pair(ab.x, ab.y, rope_cs(rp, j0 + u, rt, rh, rw));
-        w[u] = pack_bf16x2(t.x, t.y);
-      }
-      *p = x;
+  for (int i = 0; i < M; ++i) x[i] = ld_shared_u4(arow + (static_cast<uint32_t>(((c0 + i) & 7) ^ r7) << 4));
+#pragma unroll
+  for (int i = 0; i < M; ++i)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = 4 * (c0 + i) + u;
+      if constexpr (kSmem)
+        cs[i][u] = ld_shared_f2((j < pt ? bt : (j < pth ? bh : bw)) + 8u * j);
+      else
+        cs[i][u] = __ldg((j < pt ? rt : (j < pth ? rh : rw)) + j);
     }
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(&x[i]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 ab = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+      const float2 t = turn_pair(ab.x, ab.y, cs[i][u]);
+      w[u] = pack_bf16x2(t.x, t.y);
+    }
+    st_shared_u4(arow + (static_cast<uint32_t>(((c0 + i) & 7) ^ r7) << 4), x[i]);
+  }
+}
+
+// The nca chunks (features < D) of one atom of one tile row at `arow`, logical chunks cbase ..:
+// a full atom as one straight-line group, a partial one four chunks at a time.
+template <bool kSmem>
+__device__ __forceinline__ void turn_atom(uint32_t arow, int cbase, int nca, int r7, int pt, int pth, uint32_t bt,
+                                          uint32_t bh, uint32_t bw, const float2* rt, const float2* rh,
+                                          const float2* rw) {
+  if (nca == 8) {
+    turn_group<kSmem, 8>(arow, cbase, r7, pt, pth, bt, bh, bw, rt, rh, rw);
+    return;
+  }
+  for (int c0 = 0; c0 < nca; c0 += 4) {
+    switch (nca - c0) {
+      case 1: turn_group<kSmem, 1>(arow, cbase + c0, r7, pt, pth, bt, bh, bw, rt, rh, rw); break;
+      case 2: turn_group<kSmem, 2>(arow, cbase + c0, r7, pt, pth, bt, bh, bw, rt, rh, rw); break;
+      case 3: turn_group<kSmem, 3>(arow, cbase + c0, r7, pt, pth, bt, bh, bw, rt, rh, rw); break;
+      default: turn_group<kSmem, 4>(arow, cbase + c0, r7, pt, pth, bt, bh, bw, rt, rh, rw); break;
+    }
+  }
+}
+
+// Turns the feature pairs (2p, 2p + 1) of atom `atom` (features 64 atom .. 64 atom + 63) of row r
+// of a 128-row bf16 tile of swizzle-128B atoms in place, if r < rows; row r is token n0 + r. A
+// warpgroup (128 threads, thread r owning row r) turns one atom of the whole tile: the row's
+// position (frame, grid row, column) is found once and its 16-byte chunks are independent of one
+// another. Logical chunk c of a row sits at physical chunk c ^ (r % 8), so at each step the eight
+// rows r..r+7 touch eight different chunks and a warp's 16-byte accesses are free of bank
+// conflicts. (cos, sin) come from the compact table in shared memory at `ct` when
+// rp.compact > 0, else from the table in global memory; the choice is made once, outside the loops.
+__device__ __forceinline__ void rope_tile_inplace(uint8_t* tile, int atom, int r, int n0, int rows, const RopeDev& rp,
+                                                  uint32_t ct) {
+  const int nca = min(8, rp.half / 4 - 8 * atom);  // chunks of this atom holding features < D
+  if (r >= rows || nca <= 0) return;
+  const int pt = rp.pt, pth = rp.pth;
+  const uint32_t arow = smem_u32(tile) + static_cast<uint32_t>(atom * kAtomBytes + r * 128);
+  if (rp.compact > 0) {
+    uint32_t bt, bh, bw;
+    rope_rows_smem(rp, ct, n0 + r, bt, bh, bw);
+    turn_atom<true>(arow, 8 * atom, nca, r & 7, pt, pth, bt, bh, bw, nullptr, nullptr, nullptr);
+  } else {
+    const float2 *rt, *rh, *rw;
+    rope_rows(rp, n0 + r, rt, rh, rw);
+    turn_atom<false>(arow, 8 * atom, nca, r & 7, pt, pth, 0u, 0u, 0u, rt, rh, rw);
   }
 }
 
@@ -284,33 +376,53 @@ __device__ void relu_role(uint8_t* smem, const Bars& b, long long tb, long long 
 // features) and the tile turned (the S products may read it).
 struct RopeBars {
   uint64_t* zd;   // [3] count 1 (tcgen05.commit)
-  uint64_t* rot;  // [3] count 4 (the ReLU warps)
+  uint64_t* rot;  // [3] one arrival per turning warp: 4 (one atom) or 8 (two atoms)
 };
 constexpr int kRopeBars = 2 * kStages;
 __device__ __forceinline__ RopeBars rope_bars_at(uint64_t* p) { return RopeBars{p, p + kStages}; }
-__device__ __forceinline__ void init_rope_bars(const RopeBars& rb) {
+__device__ __forceinline__ void init_rope_bars(const RopeBars& rb, bool two_atoms) {
   for (int i = 0; i < kStages; ++i) {
     mbar_init(&rb.zd[i], 1);
-    mbar_init(&rb.rot[i], 4);
+    mbar_init(&rb.rot[i], two_atoms ? 8 : 4);
   }
 }
 
-// relu_role of the rotary form: ReLU of tile k, then the turn of tile k - 1 (whose z products the
-// MMA warp issued as soon as its ReLU was done, so they have had a tile's time to retire).
-__device__ void relu_rope_role(uint8_t* smem, const Bars& b, const RopeBars& rb, const Geom& geo, long long tb,
-                               long long te, bool two_atoms, int r, int lane, const RopeDev& rp, uint32_t* status) {
+// The rotary form's (cos, sin) table is staged by the turning warps (the ReLU warps and, with two
+// atoms, the epilogue warps: nthreads 128 or 256, thread index i0), which then meet on barrier 1.
+// The table may be the previous kernel's output, hence griddepcontrol.wait first (K and V are not
+// read before it anyway).
+__device__ __forceinline__ void stage_and_sync(float2* ct, const RopeDev& rp, int i0, int nthreads) {
+  griddep_wait();
+  stage_rope_table(ct, rp, i0, nthreads);
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Turn of atom `atom` of the k-th tile (global tile t) of this CTA once its z products retired.
+__device__ __forceinline__ bool turn_k(uint8_t* smem, const RopeBars& rb, const Geom& geo, int k, long long t,
+                                       int atom, int r, int lane, const RopeDev& rp, uint32_t ct, uint32_t* status) {
+  const int s = k % kStages;
+  const bool ok = mbar_wait(&rb.zd[s], (k / kStages) & 1, status, 0x0240u | s);
+  if (!warp_all(ok)) return false;
+  const TileCoord c = tile_coord(t, geo);
+  rope_tile_inplace(smem + s * kStageBytes, atom, r, c.blk * geo.L + c.tok0, c.rows, rp, ct);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&rb.rot[s]);
+  return true;
+}
+
+// relu_role of the rotary form: ReLU of tile k, then (once the MMA warp's z products of the
+// unturned tile retired) the turn of its atom 0; the epilogue warps turn atom 1.
+// The kernel's Geom and RopeDev are copied into registers here: read through references into the
+// parameter space they would be generic loads of long latency on the turn's critical path.
+__device__ void relu_rope_role(uint8_t* smem, const Bars& b, const RopeBars& rb, const Geom& geo_p, long long tb,
+                               long long te, bool two_atoms, int r, int lane, const RopeDev& rp_p, float2* ct,
+                               uint32_t* status) {
+  const Geom geo = geo_p;
+  const RopeDev rp = rp_p;
   const int nchunks = (two_atoms ? kKBytes : kAtomBytes) / 16;
-  const auto turn = [&](int k, long long t) -> bool {
-    const int s = k % kStages;
-    const bool ok = mbar_wait(&rb.zd[s], (k / kStages) & 1, status, 0x0240u | s);
-    if (!warp_all(ok)) return false;
-    const TileCoord c = tile_coord(t, geo);
-    rope_tile_inplace(smem + s * kStageBytes, two_atoms ? 2 : 1, r, c.blk * geo.L + c.tok0, c.rows, rp);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&rb.rot[s]);
-    return true;
-  };
+  stage_and_sync(ct, rp, two_atoms ? 128 + r : r, two_atoms ? 256 : 128);
+  const uint32_t cta = smem_u32(ct);
   int k = 0;
   for (long long t = tb; t < te; ++t, ++k) {
     const int s = k % kStages;
@@ -320,10 +432,17 @@ __device__ void relu_rope_role(uint8_t* smem, const Bars& b, const RopeBars& rb,
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&b.relu[s]);
-    if (k > 0 && !turn(k - 1, t - 1)) return;
+    if (!turn_k(smem, rb, geo, k, t, 0, r, lane, rp, cta, status)) return;
   }
-  if (k > 0) turn(k - 1, te - 1);
 }
+
+// What the epilogue warps of the rotary form turn (atom 1 of every tile, with two atoms).
+struct TurnCtx {
+  uint8_t* smem;
+  RopeBars rb;
+  const RopeDev* rp;
+  float2* ct;
+};
 
 template <bool kRope>
 __device__ void mma_issue(uint8_t* smem, const Bars& b, const Geom& geo, long long tb, long long te, uint32_t tmem,
@@ -388,12 +507,23 @@ __device__ __forceinline__ void mma_role(uint8_t* smem, const Bars& b, const Geo
 // and records which CTAs hold a segment's first and last tile.
 // With `slot_ready`, every flushed slot is then published for other CTAs (value `tag`): the four
 // warps meet on the CTA barrier `flushed` (count 4) and warp 0 releases the slot's flag.
+// With `tc` (rotary form, two atoms) the four warps first turn atom 1 of each tile, in order.
 __device__ void epilogue_role(const Bars& b, const Geom& geo, long long tb, long long te, uint32_t tmem, int g,
                               int warp, int lane, float* __restrict__ partials, int2* __restrict__ segcta,
-                              uint64_t* slot_ready, uint64_t* flushed, uint64_t tag, uint32_t* status) {
+                              uint64_t* slot_ready, uint64_t* flushed, uint64_t tag, uint32_t* status,
+                              const TurnCtx* tc = nullptr) {
   const int d = warp * 32 + lane;
   int j = 0;
+  RopeDev rp{};
+  uint32_t cta = 0;
+  if (tc != nullptr) {
+    rp = *tc->rp;
+    stage_and_sync(tc->ct, rp, d, 256);
+    cta = smem_u32(tc->ct);
+  }
   for (long long t = tb; t < te; ++t) {
+    if (tc != nullptr && !turn_k(tc->smem, tc->rb, geo, static_cast<int>(t - tb), t, 1, d, lane, rp, cta, status))
+      break;
     const TileCoord c = tile_coord(t, geo);
     if (!(c.last || t == te - 1)) continue;
     const int a = j & 1;
@@ -600,14 +730,14 @@ __device__ void produce(uint8_t* smem, const Bars& b, const Maps4& m, const Geom
 // Rotary form only: per stage, the denominator products of a Q tile retired, and the tile turned.
 struct RopeBars {
   uint64_t* zd;   // [3] count 1 (tcgen05.commit)
-  uint64_t* rot;  // [3] count 4 (the ReLU warps)
+  uint64_t* rot;  // [3] one arrival per turning warp: 4 (one atom) or 8 (two atoms)
 };
 constexpr int kRopeBars = 2 * kStages;
 __device__ __forceinline__ RopeBars rope_bars_at(uint64_t* p) { return RopeBars{p, p + kStages}; }
-__device__ __forceinline__ void init_rope_bars(const RopeBars& rb) {
+__device__ __forceinline__ void init_rope_bars(const RopeBars& rb, bool two_atoms) {
   for (int i = 0; i < kStages; ++i) {
     mbar_init(&rb.zd[i], 1);
-    mbar_init(&rb.rot[i], 4);
+    mbar_init(&rb.rot[i], two_atoms ? 8 : 4);
   }
 }
 
@@ -798,31 +928,49 @@ __device__ void relu_epi_role(uint8_t* smem, const Staging& sg, const Bars& b, c
   if (two_atoms && lane == 0) bulk_wait_all();
 }
 
-// Turn of the k-th Q tile once its denominator products retired. Returns 1, or -1 if the grid failed.
-__device__ __forceinline__ int turn_q(uint8_t* smem, const RopeBars& rb, const Geom& geo, const Seq& sq, long long k,
-                                      bool two_atoms, int r, int lane, const RopeDev& rp, uint32_t* status) {
+// Turn of atom `atom` of the k-th Q tile once its denominator products retired. Returns 1, 0 when
+// tile k is the end of the sequence (checked for atom 1, whose turners run ahead of the tiles they
+// have seen), -1 if the grid failed.
+__device__ __forceinline__ int turn_q(uint8_t* smem, const Bars& b, const RopeBars& rb, const Geom& geo, const Seq& sq,
+                                      long long k, int atom, int r, int lane, const RopeDev& rp, uint32_t ct,
+                                      uint32_t* status) {
   const int s = static_cast<int>(k % kStages);
-  const bool ok = mbar_wait(&rb.zd[s], static_cast<uint32_t>((k / kStages) & 1), status, 0x1240u | s);
+  const uint32_t ph = static_cast<uint32_t>((k / kStages) & 1);
+  if (atom == 1) {
+    const bool ok = mbar_wait(&b.qfull[s], ph, status, 0x1250u | s);
+    if (!warp_all(ok)) return -1;
+    if (sq.ring[k % kRing].x < 0) return 0;
+  }
+  const bool ok = mbar_wait(&rb.zd[s], ph, status, 0x1240u | s);
   if (!warp_all(ok)) return -1;
   const volatile int4* ent = sq.ring + (k % kRing);
   const int blk = ent->z, tok0 = ent->w;
   const int blen = blk == geo.nblk - 1 ? geo.Llast : geo.L;
-  rope_tile_inplace(smem + s * kQBytes, two_atoms ? 2 : 1, r, blk * geo.L + tok0, min(kTile, blen - tok0), rp);
+  rope_tile_inplace(smem + s * kQBytes, atom, r, blk * geo.L + tok0, min(kTile, blen - tok0), rp, ct);
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) mbar_arrive(&rb.rot[s]);
   return 1;
 }
 
-// relu_epi_role of the rotary form: ReLU of tile k + kStages and the turn of tile k + kStages - 1
-// after the epilogue of tile k (one tile of lag between ReLU and turn, so that the denominator
-// products have retired). The turn of tile k + 2 waits for the MMA warp's denominator products,
-// which wait for the accumulator that the epilogue of tile k released, so the order cannot
-// deadlock; at the end of the sequence every ReLU'd tile is turned.
+// relu_epi_role of the rotary form: ReLU of tile k + kStages and the turn of atom 0 of tile
+// k + kStages - 1 after the epilogue of tile k (one tile of lag between ReLU and turn, so that the
+// denominator products have retired). The turn of tile k + 2 waits for the MMA warp's denominator
+// products, which wait for the accumulator that the epilogue of tile k released, so the order
+// cannot deadlock; at the end of the sequence every ReLU'd tile is turned. With two atoms the
+// epilogue warps turn atom 1 (epi_turn_role).
+// `ct`: the compact (cos, sin) table's shared-memory area, staged by the turning warps once the
+// scan grid has finished (nothing can be turned before: the first numerator products need its
+// prefix anyway).
+// Geom and RopeDev are copied into registers, as in the state kernel's relu_rope_role.
 __device__ void relu_rot_epi_role(uint8_t* smem, const Staging& sg, const Bars& b, const RopeBars& rb, const Maps4& m,
-                                  const Geom& geo, const Seq& sq, bool two_atoms, uint32_t tmem, int warp, int lane,
-                                  float eps, const RopeDev& rp, uint32_t* status) {
+                                  const Geom& geo_p, const Seq& sq, bool two_atoms, uint32_t tmem, int warp, int lane,
+                                  float eps, const RopeDev& rp_p, float2* ct, uint32_t* status) {
+  const Geom geo = geo_p;
+  const RopeDev rp = rp_p;
   const int r = static_cast<int>(threadIdx.x) - 128;
+  st::stage_and_sync(ct, rp, two_atoms ? 128 + r : r, two_atoms ? 256 : 128);
+  const uint32_t cta = smem_u32(ct);
   long long kr = 0, kq = 0;  // tiles ReLU'd, tiles turned
   int rs = 1;                // 1 more tiles, 0 sequence ended, -1 failed
   const auto relu_next = [&]() {
@@ -833,7 +981,7 @@ __device__ void relu_rot_epi_role(uint8_t* smem, const Staging& sg, const Bars& 
   };
   const auto turn_upto = [&](long long upto) -> bool {
     for (; kq < kr && kq < upto; ++kq)
-      if (turn_q(smem, rb, geo, sq, kq, two_atoms, r, lane, rp, status) < 0) return false;
+      if (turn_q(smem, b, rb, geo, sq, kq, 0, r, lane, rp, cta, status) < 0) return false;
     return true;
   };
   for (int i = 0; i < kStages; ++i) {
@@ -851,6 +999,32 @@ __device__ void relu_rot_epi_role(uint8_t* smem, const Staging& sg, const Bars& 
     if (rs < 0 || !turn_upto(rs == 0 ? kr : k + kStages)) break;
   }
   if (two_atoms && lane == 0) bulk_wait_all();
+}
+
+// Warps 0-3 of the rotary form with two atoms: the epilogue of output columns 0..63 of tile k, then
+// the turn of atom 1 of tile k + 2 (the same place in the order as the ReLU warps' turn of atom 0;
+// tiles 0 and 1 are turned first).
+__device__ void epi_turn_role(uint8_t* smem, const Staging& sg, const Bars& b, const RopeBars& rb, const Maps4& m,
+                              const Geom& geo_p, const Seq& sq, uint32_t tmem, int warp, int lane, float eps,
+                              const RopeDev& rp_p, float2* ct, uint32_t* status) {
+  const Geom geo = geo_p;
+  const RopeDev rp = rp_p;
+  const int r = static_cast<int>(threadIdx.x);
+  st::stage_and_sync(ct, rp, r, 256);
+  const uint32_t cta = smem_u32(ct);
+  long long kq = 0;
+  int ts = 1;  // 1 more tiles, 0 end of the sequence seen, -1 failed
+  const auto turn_upto = [&](long long upto) {
+    for (; ts > 0 && kq < upto; ++kq) ts = turn_q(smem, b, rb, geo, sq, kq, 1, r, lane, rp, cta, status);
+    return ts >= 0;
+  };
+  if (turn_upto(2)) {
+    for (long long k = 0;; ++k) {
+      if (epilogue_tile(sg, b, m, geo, sq, k, tmem, warp & 3, 0, lane, eps, status) <= 0) break;
+      if (!turn_upto(k + 3)) break;
+    }
+  }
+  if (lane == 0) bulk_wait_all();
 }
 }  // namespace ot
 
@@ -885,6 +1059,11 @@ __device__ __forceinline__ void persistent_teardown(uint32_t tmem, int warp) {
 // ------------------------------------------------------------------------------------------
 constexpr int kStateSmem = st::kRegionBytes + 1024 + 256 + 1024;   // region, barriers, alignment slack
 constexpr int kOutSmem = ot::kRegionBytes + 1024 + 512 + 1024;
+// rotary form: the compact (cos, sin) table after the barrier area
+constexpr int kRopeTableBytes = kRopeSmemEntries * 8;
+constexpr int kStateSmemRope = kStateSmem + kRopeTableBytes;
+constexpr int kOutSmemRope = kOutSmem + kRopeTableBytes;
+static_assert(kStateSmemRope <= 232448 && kOutSmemRope <= 232448, "227 KB of shared memory per CTA");
 // barrier areas (512 B): the barriers, the TMEM slot, then the 16-byte aligned tile ring
 static_assert((ot::kNumBars + 2) * 8 + ot::kRingBytes <= 512, "output kernel barrier area");
 static_assert((st::kNumBars + ot::kNumBars + 2) * 8 + ot::kRingBytes <= 512, "single-launch barrier area");
@@ -913,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Maps4 m{&k_main, &k_last, &v_main, &v_last};
   if (threadIdx.x == 0) {
     st::init_bars(b);
-    if (kRope) st::init_rope_bars(rb);
+    if (kRope) st::init_rope_bars(rb, two_atoms);
     fence_mbar_init();
   }
   st::init_smem(smem, two_atoms, kThreads);
@@ -924,13 +1103,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) st::produce(smem, b, m, geo, tb, te, two_atoms, true, status);
   } else if (warp >= 4 && warp < 8) {
     if constexpr (kRope)
-      st::relu_rope_role(smem, b, rb, geo, tb, te, two_atoms, threadIdx.x - 128, lane, rp, status);
+      st::relu_rope_role(smem, b, rb, geo, tb, te, two_atoms, threadIdx.x - 128, lane, rp,
+                         reinterpret_cast<float2*>(smem + st::kRegionBytes + 256), status);
     else
       st::relu_role(smem, b, tb, te, two_atoms, threadIdx.x - 128, lane, status);
   } else if (warp == kWarpMma) {
     if (lane == 0) st::mma_issue<kRope>(smem, b, geo, tb, te, tmem, status, &rb);
   } else {
-    st::epilogue_role(b, geo, tb, te, tmem, g, warp, lane, partials, segcta, nullptr, nullptr, 0, status);
+    const st::TurnCtx tc{smem, rb, &rp, reinterpret_cast<float2*>(smem + st::kRegionBytes + 256)};
+    st::epilogue_role(b, geo, tb, te, tmem, g, warp, lane, partials, segcta, nullptr, nullptr, 0, status,
+                      kRope && two_atoms ? &tc : nullptr);
   }
   persistent_teardown(tmem, warp);
 }
@@ -958,7 +1140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Maps4 m{&q_main, &q_last, &o_main, &o_last};
   if (threadIdx.x == 0) {
     ot::init_bars(b, two_atoms);
-    if (kRope) ot::init_rope_bars(rb);
+    if (kRope) ot::init_rope_bars(rb, two_atoms);
     fence_mbar_init();
   }
   if (warp == kWarpProducer && lane == 0) prefetch_maps(m);
@@ -973,12 +1155,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4 && warp < 8) {
     if constexpr (kRope)
       ot::relu_rot_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, rb, m, geo, sq, two_atoms, tmem, warp, lane,
-                            eps, rp, status);
+                            eps, rp, reinterpret_cast<float2*>(smem + ot::kRegionBytes + 512), status);
     else
       ot::relu_epi_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, 0, two_atoms, tmem, warp, lane, eps,
                         status);
   } else if (warp == kWarpMma) {
     if (lane == 0) ot::mma_issue<kRope>(smem, b, geo, sq, two_atoms, tmem, status, &rb);
+  } else if (kRope && two_atoms) {
+    ot::epi_turn_role(smem, ot::Staging{smem + ot::kOOff, 1}, b, rb, m, geo, sq, tmem, warp, lane, eps, rp,
+                      reinterpret_cast<float2*>(smem + ot::kRegionBytes + 512), status);
   } else {
     ot::epilogue_role(ot::Staging{smem + ot::kOOff, 1}, b, m, geo, sq, tmem, warp, lane, eps, status);
   }
@@ -2214,9 +2399,9 @@ cudaError_t set_kernel_attributes() {
   cudaError_t e;
   e = cudaFuncSetAttribute(state_bf16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(state_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+  e = cudaFuncSetAttribute(state_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmemRope);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(out_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+  e = cudaFuncSetAttribute(out_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmemRope);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(fused_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fu::kSmem);
   if (e != cudaSuccess) return e;
@@ -2234,7 +2419,7 @@ cudaError_t set_kernel_attributes() {
 cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom& g, float* partials, int2* segcta,
                               uint32_t* status, cudaStream_t s, const RopeDev* rope) {
   if (rope != nullptr)
-    return launch_pdl(state_bf16_kernel<true>, dim3(g.G), dim3(kThreads), kStateSmem, s, k.main, k.last, v.main,
+    return launch_pdl(state_bf16_kernel<true>, dim3(g.G), dim3(kThreads), kStateSmemRope, s, k.main, k.last, v.main,
                       v.last, g, partials, segcta, status, *rope);
   return launch_pdl(state_bf16_kernel<false>, dim3(g.G), dim3(kThreads), kStateSmem, s, k.main, k.last, v.main,
                     v.last, g, partials, segcta, status, RopeDev{});
@@ -2243,7 +2428,8 @@ cudaError_t launch_state_bf16(const BlockMaps& k, const BlockMaps& v, const Geom
 cudaError_t launch_out_bf16(const BlockMaps& q, const BlockMaps& o, const Geom& g, const void* ptiles, float eps,
                             uint32_t* status, cudaStream_t s, const RopeDev* rope) {
   if (rope != nullptr)
-    return launch_pdl(out_bf16_kernel<true>, dim3(g.G), dim3(kThreads), kOutSmem, s, q.main, q.last, o.main, o.last,
+    return launch_pdl(out_bf16_kernel<true>, dim3(g.G), dim3(kThreads), kOutSmemRope, s, q.main, q.last, o.main,
+                      o.last,
                       g, static_cast<const uint8_t*>(ptiles), eps, status, *rope);
   return launch_pdl(out_bf16_kernel<false>, dim3(g.G), dim3(kThreads), kOutSmem, s, q.main, q.last, o.main, o.last,
                     g, static_cast<const uint8_t*>(ptiles), eps, status, RopeDev{});
