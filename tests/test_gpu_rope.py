@@ -69,13 +69,13 @@ def test_table_matches_the_oracle_angles(sv, D, frames, height, width):
     assert np.max(np.abs(got[..., 1] - np.sin(ang))) < 1e-6
 
 
-def run_rope(sv, dtype, shape, L, height, width, frame0=0, with_cache=True, seed=0):
+def run_rope(sv, dtype, shape, L, height, width, frame0=0, with_cache=True, seed=0, pairs=None):
     B, H, N, D = shape
     st = draw_qkv(shape, seed, dtype)
     q, k, v = (to_f64(x, dtype) for x in st)
     hw = height * width
     frames = frame0 + (N - 1) // hw + 1
-    pairs = R.default_pairs(D)
+    pairs = R.default_pairs(D) if pairs is None else pairs
     tab = sv.sv_rope3d_table(frames, height, width, D, pairs)
     S_in, z_in = cache_in(B, H, D, seed + 1) if with_cache else (None, None)
     S_out = torch.zeros(B, H, D, D, device="cuda")
@@ -119,6 +119,22 @@ def test_bf16_matches_oracle(sv, B, H, N, D, L, height, width):
 def test_f32_matches_oracle(sv, B, H, N, D, L, height, width):
     got, ref = run_rope(sv, "f32", (B, H, N, D), L, height, width, frame0=1, seed=N)
     check(got, ref, "f32")
+
+
+def test_bf16_table_beyond_shared_memory(sv):
+    # 4 x 4 tokens per frame: the call touches 188 frames, so the compact (cos, sin) table would
+    # need 188 * 22 + 4 * 21 + 4 * 21 = 4304 entries, more than the kernels stage in shared memory
+    # (3072): they read the table in global memory instead
+    got, ref = run_rope(sv, "bf16", (1, 2, 3000, 128), 800, 4, 4, seed=31)
+    check(got, ref, "bf16")
+
+
+@pytest.mark.parametrize("dtype,D,pairs", [("bf16", 128, (32, 0, 32)), ("bf16", 64, (0, 16, 16)),
+                                           ("bf16", 112, (56, 0, 0)), ("f32", 32, (0, 0, 16))])
+def test_caller_given_pair_splits(sv, dtype, D, pairs):
+    # empty groups, and all pairs on one axis
+    got, ref = run_rope(sv, dtype, (1, 2, 600, D), 200, 5, 6, frame0=3, seed=D, pairs=pairs)
+    check(got, ref, dtype)
 
 
 def test_bf16_without_incoming_cache(sv):
