@@ -422,7 +422,7 @@ def _cpu_model():
     return platform.processor() or "unknown"
 
 
-def time_workload(name, passes: int, dev_index: int = 0):
+def time_workload(name, passes: int, dev_index: int = 0, heads: int | None = None):
     """Device time of one of the other configurations, as a dict for the bench line. Every call of a
     pass gets distinct inputs (torch's seeded CUDA generator, seed 0), so L2 never holds a call's
     inputs from an earlier call. Eager: CUDA events around each call issued from Python through the
@@ -433,6 +433,9 @@ def time_workload(name, passes: int, dev_index: int = 0):
     import block_causal_linear_relu_b200 as sv
 
     desc, b, h, n, d, blen, kind, reps = EXTRA_WORKLOADS[name]
+    if heads is not None:  # a smaller case of the same workload, for profiling captures only
+        h = heads
+        desc += f" (heads overridden to {heads}: not the configuration)"
     dev = torch.device("cuda", dev_index)
     hbm_gbs, _, _, _ = peaks()
     gen = torch.Generator(device=dev)
@@ -663,7 +666,7 @@ def run_extra(args, name):
 
     torch.cuda.set_device(0)
     sv.load()
-    r = time_workload(name, max(1, args.steps // EXTRA_WORKLOADS[name][-1]))
+    r = time_workload(name, max(1, args.steps // EXTRA_WORKLOADS[name][-1]), heads=args.heads)
     line = {"metric": METRIC, "value": r["graph"]["value"], "unit": UNIT, "n_gpus": 1, "workload": name,
             "impl": "ours", "dtype": "bf16", **r}
     print(json.dumps(line), flush=True)
