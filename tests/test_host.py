@@ -106,6 +106,19 @@ def test_rope_arguments_are_checked_before_any_launch(lib):
     assert call(SvRope3d(**good), D=100) == 2  # bf16 D must be a multiple of 8 (checked first)
 
 
+def test_binding_rope_helpers(lib):
+    # the binding's table size and default pair split (host only); the split agrees with the oracle's
+    import block_causal_linear_relu_b200 as sv
+    from oracle import rope as R
+
+    assert sv.sv_rope3d_table_bytes(60, 23, 40, 128) == (60 + 23 + 40) * 64 * 8
+    with pytest.raises(sv.SvError, match="even"):
+        sv.sv_rope3d_table_bytes(60, 23, 40, 127)
+    for D in (8, 24, 64, 112, 128):
+        assert sv.rope_pairs(D) == R.default_pairs(D)
+        assert 2 * sum(sv.rope_pairs(D)) == D
+
+
 def test_binding_rejects_bad_tensors_before_the_library():
     # the binding's single pass of checks: host tensors, wrong rank, mismatched shape or dtype and
     # non-contiguous tensors raise before any library or CUDA call
