@@ -140,6 +140,53 @@ def oracle_rate(q, k, v, budget_s: float, max_heads: int | None = None):
     return done * N / dt, done, N, dt
 
 
+def oracle_rates_other(budget_s: float):
+    """The fp64 oracle (as it stands) on bounded samples of the other configurations, on the host
+    cores, each sample repeated until budget_s elapse (at least once). Rates in the units of those
+    configurations' GPU figures; a reported baseline, not a target."""
+    import oracle
+    from oracle import rope as R
+    from block_causal_linear_relu_b200.inputs import draw_conv, draw_proj, draw_qkv, to_f64
+
+    def run(fn):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= budget_s:
+                return n, dt
+
+    def attn_line(name, shape, fn, what):
+        q, k, v = (to_f64(x, "bf16") for x in draw_qkv(shape, 0, "bf16"))
+        n, dt = run(lambda: fn(q, k, v))
+        out[name] = {"value": n * shape[1] * shape[2] / dt, "unit": UNIT,
+                     "sample": f"fp64 numpy oracle, {what}, {n} run(s), {dt:.1f} s"}
+
+    out = {}
+    attn_line("480p_bidir", (1, 1, 8190, 112), lambda q, k, v: oracle.linattn_fwd(q, k, v, EPS),
+              "one head of the 480p bidirectional layer [1, 1, 8190, 112]")
+    S0, z0 = np.zeros((1, 1, D, D)), np.zeros((1, 1, D))
+    attn_line("720p_stream", (1, 1, L, D), lambda q, k, v: oracle.cache_step(q, k, v, S0, z0, EPS),
+              "one head of one streaming block [1, 1, 2760, 128] through the cache")
+    ang = R.rope3d_angles(R.token_positions(N, 23, 40), R.default_pairs(D))
+    attn_line("720p_prefill_rope", (1, 1, N, D), lambda q, k, v: R.block_causal_attn_rope(q, k, v, L, EPS, ang),
+              "one head of the 720p prefill with 3D RoPE [1, 1, 55200, 128], blocks of 2760")
+    xs, w, bias = draw_conv((1, 60, 920, 64), 0, "bf16")
+    xf = to_f64(xs, "bf16")
+    n, dt = run(lambda: oracle.temporal_conv_block_causal(xf, w, bias, 3))
+    out["720p_temporal_conv"] = {"value": n * 2 * xf.size * 2 / dt / 1e9, "unit": "GB/s (bf16 bytes read + written)",
+                                 "sample": f"fp64 numpy oracle, 64 of the 2560 channels of x [1, 60, 920, C], "
+                                           f"blocks of 3 frames, {n} run(s), {dt:.1f} s"}
+    xp, wp = draw_proj((1, 512, 2560), 3 * 2560, 0)
+    xpf, wpf = to_f64(xp, "bf16"), to_f64(wp, "bf16")
+    n, dt = run(lambda: oracle.qkv_projection(xpf, wpf, 20, 128))
+    out["sv2_projections"] = {"value": n * 2 * 512 * 2560 * 7680 / dt / 1e12, "unit": "TFLOP/s",
+                              "sample": f"fp64 numpy oracle, the Q/K/V projection of 512 of the 20240 rows "
+                                        f"[512 x 2560] x [2560 x 7680], {n} run(s), {dt:.1f} s"}
+    return out
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
@@ -367,6 +414,8 @@ def run_ours(args, rank: int, world: int):
         cpu = {"value": rate, "unit": UNIT, "cores": _blas_threads(), "cpu_model": _cpu_model(), "kind": "oracle",
                "sample": f"fp64 numpy oracle (state form), {nh} heads x {ntok} tokens cycling over this "
                          f"workload's {H} heads ({nh / H:.1f} passes), {secs:.1f} s"}
+        if not args.no_extras:  # the oracle beside the other configurations' GPU figures
+            cpu["other_configs"] = oracle_rates_other(1.5)
     extras = None
     if world == 1 and not args.no_extras:
         extras = {}

@@ -119,6 +119,16 @@ def test_binding_rope_helpers(lib):
         assert 2 * sum(sv.rope_pairs(D)) == D
 
 
+def test_oracle_rates_of_the_other_configurations():
+    # the bench's CPU-baseline leg for the other configurations: every sample runs and gives a rate
+    import bench
+
+    r = bench.oracle_rates_other(0.0)
+    assert set(r) == {"480p_bidir", "720p_stream", "720p_prefill_rope", "720p_temporal_conv", "sv2_projections"}
+    for v in r.values():
+        assert v["value"] > 0 and v["unit"] and "1 run(s)" in v["sample"]
+
+
 def test_binding_rejects_bad_tensors_before_the_library():
     # the binding's single pass of checks: host tensors, wrong rank, mismatched shape or dtype and
     # non-contiguous tensors raise before any library or CUDA call
