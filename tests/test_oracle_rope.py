@@ -72,6 +72,18 @@ def test_matches_bruteforce_with_dense_rotations(blen):
     assert oracle.max_rel_err(o, R.bruteforce_rope(q, k, v, blen, EPS, ang)) < 1e-12
 
 
+@pytest.mark.parametrize("blen,pairs", [(12, (2, 2, 2)), (30, (1, 0, 5)), (1000, (6, 0, 0))])
+def test_matches_c_bruteforce_through_relative_angles(blen, pairs):
+    # a second brute force, in plain C, that never turns a vector: each pair's score is written
+    # with the cosine and sine of the angle difference (oracle/bruteforce.c)
+    from oracle.bruteforce import bruteforce_rope_c
+
+    q, k, v = _qkv((2, 1, 60, 12), 23)
+    ang = R.rope3d_angles(R.token_positions(60, 2, 5, frame0=4), pairs)
+    o, _, _ = R.block_causal_attn_rope(q, k, v, blen, EPS, ang)
+    assert oracle.max_rel_err(o, bruteforce_rope_c(q, k, v, blen, EPS, ang)) < 1e-12
+
+
 @pytest.mark.parametrize("blen", [18, 1000])
 def test_output_depends_on_relative_positions_only(blen):
     # every score of the numerator is phi(q_i)^T R(angle_j - angle_i) phi(k_j): moving every token
@@ -175,6 +187,8 @@ def test_planted_mistake_is_caught(kind):
     ref = R.bruteforce_rope(q, k, v, 12, EPS, ang)
     assert oracle.max_rel_err(_mutant("none", q, k, v, 12, EPS, ang), ref) < 1e-12
     assert oracle.max_rel_err(_mutant(kind, q, k, v, 12, EPS, ang), ref) > 1e-3
+    from oracle.bruteforce import bruteforce_rope_c
+    assert oracle.max_rel_err(_mutant(kind, q, k, v, 12, EPS, ang), bruteforce_rope_c(q, k, v, 12, EPS, ang)) > 1e-3
     qh, kh, vh, angh = _hand_case()
     good = (13 + 7 * math.cos(1.0)) / 8  # token 3 (frame 1, column 1), bidirectional
     if kind != "half_split_pairs":  # the hand case's features sit on the interleaved pairs only
