@@ -33,11 +33,12 @@ the plainest one that keeps the rest of the method intact:
 
 Pins (tests/test_oracle_rope.py): zero angles reduce it to the pinned plain oracle; an
 independent brute force builds every rotation as a dense block-diagonal D x D matrix and the
-explicit masked N x N score matrices; a second one, in plain C (bruteforce.c), never turns a vector
-and writes each pair's score through the cosine and sine of the angle difference; shifting frame0 leaves the bidirectional output unchanged
-(relative positions); a D = 4 case whose angles are whole radians checked against closed forms;
-streaming through the cache equals the prefill; planted mistakes (rotated denominator, q turned
-the other way, half-split pairs) each fail a pin. The pages fix none of this form, so parity of
+explicit masked N x N score matrices; a second one, in plain C (bruteforce.c), never turns a
+vector and writes each pair's score through the cosine and sine of the angle difference;
+shifting frame0 leaves the bidirectional output unchanged (relative positions); a D = 4 case
+whose angles are whole radians checked against closed forms; streaming through the cache equals
+the prefill; planted mistakes (rotated denominator, q turned the other way, half-split pairs)
+each fail a pin. The pages fix none of this form, so parity of
 this function is pinned to the mathematics of the reading above, not to the pages ("parity
 unpinned" with respect to the pages).
 """
